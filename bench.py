@@ -1,0 +1,515 @@
+"""Benchmark: MoE dispatch / combine on B200, V3-shaped workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = the whole hot path over one batch: layout -> FP8 dispatch (bf16
+x quantised to e4m3 with 1x128 scales) -> BF16 combine, on the workload of
+the DeepEP V2 README, section "Performance" (8192 tokens, hidden 7168,
+top-8 of 256 experts in 8 segments, expert_alignment 128), synthetic seeded
+inputs.  Prints ONE JSON line on rank 0.
+
+value = algorithmic bytes of the step (below) / device time of the step,
+        summed over ranks / max-over-ranks time (weak scaling: every rank
+        runs its own batch; there is no exchange on this path).
+Algorithmic bytes (per step, from the layout the step produced):
+  layout   : topk_idx + topk_weights read, slot_map + 3 per-row arrays written
+  dispatch : x read once (T*H*2) + slot_map read + for each valid slot one
+             e4m3 row (H) and its scales (H/128*4) written + for each padding
+             row H + H/128*4 zero bytes written
+  combine  : for each valid slot one bf16 row of y read (H*2) + slot_map and
+             weights read + the bf16 output written (T*H*2)
+The step touches ~1.8 GB, far more than the 126 MB L2, so no L2 flush is
+needed between steps.
+
+--impl reference times the CPU oracle (the only other implementation of
+this path; single-threaded C) on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "dispatch & combine GB/s and % of B200 HBM peak (V3 shape); decode µs/call"
+WORKLOAD = "v3"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=WORKLOAD, choices=sorted(W.WORKLOADS))
+    p.add_argument("--decode-pairs", type=int, default=256)
+    p.add_argument("--decode-replays", type=int, default=20)
+    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------ byte counts
+
+def step_bytes(w: W.Workload, T: int, V: int, P: int, R: int) -> dict:
+    """Algorithmic bytes of one layout / dispatch / combine, given the valid
+    slot count V, padding rows P and total rows R of the layout."""
+    H, k = w.H, w.k
+    B = H // 128
+    layout = T * k * 8 + T * k * 4 + T * k * 4 + R * 12
+    if w.x_mode == "fp8_quant":
+        dispatch = T * H * 2 + T * k * 4 + V * (H + B * 4) + P * (H + B * 4)
+    else:
+        dispatch = T * H * 2 + T * k * 4 + (V + P) * H * 2
+    combine = V * H * 2 + T * k * 8 + T * H * 2
+    return {"layout": layout, "dispatch": dispatch, "combine": combine}
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_id: str | None):
+        self.proc = None
+        self.device_id = device_id
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.device_id is not None:
+            cmd += ["-i", self.device_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def nvsmi_device_id(dev) -> str | None:
+    import torch
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        return vis.split(",")[dev.index or 0] if vis else str(dev.index or 0)
+
+
+# ----------------------------------------------------------- ncu traffic
+
+def combine_traffic():
+    """Per-launch DRAM bytes of the combine kernel from the committed ncu
+    summary, if that summary was taken on the current combine source."""
+    src = os.path.join(ROOT, "combine_ep_get_06_b200", "csrc", "combine.cu")
+    summ = os.path.join(ROOT, "profiles", "combine_kernel_v3.md")
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        text = open(summ).read()
+    except OSError:
+        return None
+    m_sha = re.search(r"combine\.cu sha256\[:16\]:\s*`?([0-9a-f]{16})", text)
+    m_tr = re.search(r"traffic per launch \(bytes\):\s*([0-9]+)", text)
+    if m_sha and m_tr and m_sha.group(1) == sha:
+        return int(m_tr.group(1))
+    return None
+
+
+# ------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, dev):
+    import torch
+    import torch.distributed as dist
+
+    import combine_ep_get_06_b200 as ep
+
+    w = W.WORKLOADS[args.workload]
+    inp = W.make_inputs(w, seed=rank)
+    y_np = W.make_y(w, seed=rank)
+    T, k, H = w.T, w.k, w.H
+
+    def bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    x = bf16(inp["x"])
+    y = bf16(y_np)
+    idx = torch.from_numpy(inp["topk_idx"]).to(dev)
+    wts = torch.from_numpy(inp["topk_weights"]).to(dev)
+    fp8 = w.x_mode == "fp8_quant"
+    handle = ep.EPHandle(T, k, w.E, w.S, w.align, device=dev)
+    rows = handle.max_recv_rows
+    recv_idx = torch.empty(rows, dtype=torch.int32, device=dev)
+    recv_w = torch.empty(rows, dtype=torch.float32, device=dev)
+    if fp8:
+        recv_x = torch.empty(rows, H, dtype=torch.float8_e4m3fn, device=dev)
+        recv_s = torch.empty(rows, H // 128, dtype=torch.float32, device=dev)
+    else:
+        recv_x = torch.empty(rows, H, dtype=torch.bfloat16, device=dev)
+        recv_s = None
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def layout():
+        ep.get_layout(idx, w.E, num_segments=w.S, expert_alignment=w.align, topk_weights=wts,
+                      handle=handle, recv_topk_idx=recv_idx, recv_topk_weights=recv_w)
+
+    def dispatch():
+        ep.dispatch_with_handle(x, handle, use_fp8=fp8, recv_x=recv_x, recv_scales=recv_s)
+
+    def combine():
+        ep.combine(y, handle, wts, out=out)
+
+    for _ in range(args.warmup):
+        layout(); dispatch(); combine()
+    torch.cuda.synchronize(dev)
+    V = int(handle.counts.sum())
+    P = int(handle.num_pad_rows[0])
+    R = handle.total_rows()
+    nbytes = step_bytes(w, T, V, P, R)
+    handle.check_error()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(nvsmi_device_id(dev))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    start.record(stream)
+    for i in range(K):
+        e = ev[i]
+        e[0].record(stream); layout()
+        e[1].record(stream); dispatch()
+        e[2].record(stream); combine()
+        e[3].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    total_ms = start.elapsed_time(end)
+    lay_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    dis_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    com_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+    handle.check_error()
+
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / K
+    step_total = sum(nbytes.values())
+    value = step_total * world / (ms_per_step * 1e-3) / 1e9
+    peak, peak_kind = hbm_peak()
+
+    res = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"{w.name}: T={T} hidden={H} experts={w.E} segments={w.S} "
+                               f"topk={k} alignment={w.align} x={w.x_mode}",
+                   "T": T, "hidden": H, "experts": w.E, "segments": w.S, "topk": k,
+                   "alignment": w.align, "dispatch": "bf16 -> e4m3 1x128" if fp8 else "bf16",
+                   "combine": "bf16, weighted, fp32 accumulation", "parallelism": f"replicas{world}",
+                   "l2": "no flush: each step touches ~1.8 GB, > 126 MB L2"},
+        "gpu_launches": K * (4 if handle.c.num_tokens * k > 2048 else 3),
+        "layout_us": round(lay_ms * 1e3, 2),
+        "dispatch": {"us": round(dis_ms * 1e3, 2), "bytes": nbytes["dispatch"],
+                     "gbs": round(nbytes["dispatch"] / (dis_ms * 1e-3) / 1e9, 1),
+                     "frac_of_peak": round(nbytes["dispatch"] / (dis_ms * 1e-3) / 1e9 / peak, 4),
+                     "valid_rows": V, "padding_rows": P},
+        "combine": {"us": round(com_ms * 1e3, 2), "bytes": nbytes["combine"],
+                    "gbs": round(nbytes["combine"] / (com_ms * 1e-3) / 1e9, 1),
+                    "frac_of_peak": round(nbytes["combine"] / (com_ms * 1e-3) / 1e9 / peak, 4)},
+        "clocks": clocks,
+    }
+    achieved = nbytes["combine"] / (com_ms * 1e-3) / 1e9
+    res["roofline"] = {"bound": "hbm", "kernel": "combine_kernel", "achieved": round(achieved, 1),
+                       "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                       "frac": round(achieved / peak, 4), "traffic": combine_traffic(),
+                       "algorithmic_bytes": nbytes["combine"]}
+
+    if not args.no_decode:
+        res["decode"] = run_decode(args, dev)
+    if not args.no_e2e:
+        res["e2e"] = run_e2e(args, dev, w, inp, y_np, nbytes)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w, inp, y_np)
+    return res
+
+
+def run_decode(args, dev):
+    """decode: T=128, hidden 7168, 256 experts, top-8, alignment 1, FP8
+    dispatch + BF16 combine; `pairs` layout->dispatch->combine pairs
+    captured in one CUDA graph (4 routings in turn, shared receive
+    buffers, as one layer after another would reuse them)."""
+    import torch
+
+    import combine_ep_get_06_b200 as ep
+
+    w = W.WORKLOADS["decode"]
+    n_route = 4
+    inps = [W.make_inputs(w, seed=1000 + i) for i in range(n_route)]
+
+    def bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    rows = ep.max_recv_rows(w.T, w.k, w.E, w.align)
+    y = bf16(W.make_y(w, seed=1000, rows=rows))
+    idx = [torch.from_numpy(i["topk_idx"]).to(dev) for i in inps]
+    wts = [torch.from_numpy(i["topk_weights"]).to(dev) for i in inps]
+    xs = [bf16(i["x"]) for i in inps]
+    hs = [ep.EPHandle(w.T, w.k, w.E, w.S, w.align, device=dev) for _ in range(n_route)]
+    ri = torch.empty(rows, dtype=torch.int32, device=dev)
+    rw = torch.empty(rows, dtype=torch.float32, device=dev)
+    rq = torch.empty(rows, w.H, dtype=torch.float8_e4m3fn, device=dev)
+    rs = torch.empty(rows, w.H // 128, dtype=torch.float32, device=dev)
+    out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev)
+
+    def pairs(n, cached=False):
+        for p in range(n):
+            i = p % n_route
+            if not cached:
+                ep.get_layout(idx[i], w.E, num_segments=w.S, expert_alignment=w.align,
+                              topk_weights=wts[i], handle=hs[i], recv_topk_idx=ri, recv_topk_weights=rw)
+            ep.dispatch_with_handle(xs[i], hs[i], use_fp8=True, recv_x=rq, recv_scales=rs)
+            ep.combine(y, hs[i], wts[i], out=out)
+
+    result = {"config": "decode: T=128 hidden=7168 experts=256 topk=8 alignment=1 fp8 dispatch + "
+                        "bf16 combine", "pairs_per_graph": args.decode_pairs}
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        pairs(n_route)
+    torch.cuda.current_stream(dev).wait_stream(s)
+    torch.cuda.synchronize(dev)
+    for cached in (False, True):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            pairs(args.decode_pairs, cached)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize(dev)
+        times = []
+        for _ in range(args.decode_replays):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            b.record()
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        us = statistics.median(times) * 1e3 / args.decode_pairs
+        result["cached_handle_us_per_pair" if cached else "us_per_pair"] = round(us, 3)
+        del g
+    for h in hs:
+        h.check_error()
+    return result
+
+
+def run_e2e(args, dev, w, inp, y_np, nbytes):
+    """Same metric through the public API with HOST inputs: every step
+    copies x, topk_idx, topk_weights and y from pinned host memory, runs
+    layout -> dispatch -> combine, and copies recv_x, recv_scales and the
+    combined output back to pinned host memory."""
+    import torch
+
+    import combine_ep_get_06_b200 as ep
+
+    T, k, H = w.T, w.k, w.H
+    fp8 = w.x_mode == "fp8_quant"
+    hx = torch.from_numpy(np.ascontiguousarray(inp["x"]).view(np.int16)).view(torch.bfloat16).pin_memory()
+    hi = torch.from_numpy(inp["topk_idx"]).pin_memory()
+    hw = torch.from_numpy(inp["topk_weights"]).pin_memory()
+    hy = torch.from_numpy(np.ascontiguousarray(y_np).view(np.int16)).view(torch.bfloat16).pin_memory()
+    handle = ep.EPHandle(T, k, w.E, w.S, w.align, device=dev)
+    rows = handle.max_recv_rows
+    dx = torch.empty_like(hx, device=dev)
+    di = torch.empty_like(hi, device=dev)
+    dw = torch.empty_like(hw, device=dev)
+    dy = torch.empty_like(hy, device=dev)
+    rq = torch.empty(rows, H, dtype=torch.float8_e4m3fn if fp8 else torch.bfloat16, device=dev)
+    rs = torch.empty(rows, H // 128, dtype=torch.float32, device=dev) if fp8 else None
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    h_rq = torch.empty(rq.shape, dtype=rq.dtype).pin_memory()
+    h_rs = torch.empty(rs.shape, dtype=rs.dtype).pin_memory() if fp8 else None
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = hx.numel() * 2 + hi.numel() * 8 + hw.numel() * 4 + hy.numel() * 2
+    d2h = h_rq.numel() * h_rq.element_size() + (h_rs.numel() * 4 if fp8 else 0) + h_out.numel() * 2
+
+    def step():
+        dx.copy_(hx, non_blocking=True)
+        di.copy_(hi, non_blocking=True)
+        dw.copy_(hw, non_blocking=True)
+        ep.get_layout(di, w.E, num_segments=w.S, expert_alignment=w.align, topk_weights=dw, handle=handle)
+        ep.dispatch_with_handle(dx, handle, use_fp8=fp8, recv_x=rq, recv_scales=rs)
+        h_rq.copy_(rq, non_blocking=True)
+        if fp8:
+            h_rs.copy_(rs, non_blocking=True)
+        dy.copy_(hy, non_blocking=True)
+        ep.combine(dy, handle, dw, out=out)
+        h_out.copy_(out, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.e2e_steps):
+        step()
+    b.record()
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b) / args.e2e_steps
+    total = sum(nbytes.values())
+    return {"value": round(total / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(ms, 3),
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+
+
+# ------------------------------------------------------ CPU oracle timing
+
+def time_oracle_step(w: W.Workload, inp, y_np):
+    import oracle
+
+    T = inp["x"].shape[0]
+    t0 = time.perf_counter()
+    lay = oracle.layout(inp["topk_idx"], w.E, w.S, w.align, inp["topk_weights"])
+    oracle.dispatch(lay, inp["x"], oracle.X_BF16_QUANT_FP8 if w.x_mode == "fp8_quant" else oracle.X_BF16)
+    oracle.combine(lay["slot_map"], T, w.k, y_np, inp["topk_weights"])
+    dt = time.perf_counter() - t0
+    V = int(lay["counts"].sum())
+    R = lay["R"]
+    nb = step_bytes(w, T, V, R - V, R)
+    return dt, sum(nb.values())
+
+
+def cpu_baseline(w: W.Workload, inp, y_np, reps=3):
+    runs = [time_oracle_step(w, inp, y_np) for _ in range(reps)]
+    dt = statistics.median(r[0] for r in runs)
+    nb = runs[0][1]
+    return {"value": round(nb / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"the full {w.name} workload (T={inp['x'].shape[0]}), layout+dispatch+combine, "
+                      f"median of {reps} runs ({dt:.2f} s each), single-threaded C",
+            "host_cores_available": os.cpu_count()}
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle, timed as it stands, on a bounded
+    token sample of the same workload per step (sized so that the whole
+    run stays within about two minutes)."""
+    w = W.WORKLOADS[args.workload]
+    probe_T = 64
+    inp = W.make_inputs(w, seed=0, T=probe_T)
+    y_np = W.make_y(w, seed=0, rows=W.y_rows(W.Workload(**{**w.__dict__, "T": probe_T})))
+    dt, _ = time_oracle_step(w, inp, y_np)
+    per_token = dt / probe_T
+    budget = 100.0 / max(1, args.steps + args.warmup)
+    T_s = int(max(16, min(w.T, budget / max(per_token, 1e-9))))
+    inp = W.make_inputs(w, seed=0, T=T_s)
+    y_np = W.make_y(w, seed=0, rows=W.y_rows(W.Workload(**{**w.__dict__, "T": T_s})))
+    for _ in range(args.warmup):
+        time_oracle_step(w, inp, y_np)
+    tot_t, tot_b = 0.0, 0
+    for _ in range(args.steps):
+        dt, nb = time_oracle_step(w, inp, y_np)
+        tot_t += dt
+        tot_b += nb
+    value = tot_b / tot_t / 1e9
+    sample = (f"{T_s} of the {w.T} tokens of the {w.name} workload per step (same hidden, experts, "
+              f"top-k, alignment), layout+dispatch+combine, single-threaded C oracle")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_t / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": f"{w.name}: T={w.T} hidden={w.H} experts={w.E} segments={w.S} "
+                               f"topk={w.k} alignment={w.align} x={w.x_mode}"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    try:
+        res = run_ours(args, rank, world, dev)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

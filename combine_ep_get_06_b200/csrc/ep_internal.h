@@ -1,0 +1,70 @@
+// Internal interface between the C-ABI front end (ep_api.cpp) and the
+// kernels (layout.cu, dispatch.cu, combine.cu).  Not installed.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ep.h"
+
+namespace ep {
+
+// Layout: slots are processed in chunks of whole tokens, about
+// kLayoutChunkSlots slots each, one CTA per chunk.
+constexpr int kLayoutThreads = 1024;
+constexpr int kLayoutChunkSlots = 2048;
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxTopk = 32;
+
+struct LayoutArgs {
+    const void* topk_idx;
+    const float* topk_weights;
+    int32_t* recv_topk_idx;
+    float* recv_topk_weights;
+    ep_handle h;            // by value: pointers into the caller's block
+    int32_t chunk_tokens;   // tokens per chunk
+    int32_t num_chunks;
+    int32_t* ws_hist;       // [num_chunks][E]
+    int32_t* ws_seg;        // [num_chunks][S]
+};
+
+inline int layout_chunk_tokens(int k) { return kLayoutChunkSlots / k > 0 ? kLayoutChunkSlots / k : 1; }
+inline int layout_num_chunks(int T, int k) {
+    int ct = layout_chunk_tokens(k);
+    int c = (T + ct - 1) / ct;
+    return c > 0 ? c : 1;
+}
+
+cudaError_t launch_layout(const LayoutArgs& a, bool idx_is_int64, cudaStream_t stream);
+
+struct DispatchArgs {
+    const void* x;
+    const float* x_scales;
+    void* recv_x;
+    float* recv_scales;
+    const int32_t* slot_map;
+    const int32_t* pad_rows;
+    const int32_t* num_pad_rows;
+    uint32_t* error_word;
+    int32_t T, k, H, max_rows;
+};
+
+cudaError_t launch_dispatch(const DispatchArgs& a, ep_x_mode mode, cudaStream_t stream);
+
+struct CombineArgs {
+    const void* y;
+    const float* topk_weights;       // nullable: unweighted
+    const float* recv_weights_in;    // nullable
+    float* out_weights;              // nullable
+    void* out;
+    const int32_t* slot_map;
+    uint32_t* error_word;
+    int32_t T, k, H, max_rows;
+};
+
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
+
+// Number of SMs of the current device (cached per device).
+int device_sm_count();
+
+}  // namespace ep
