@@ -325,10 +325,12 @@ def run_decode(args, dev):
     def pairs(n, cached=False):
         for p in range(n):
             i = p % n_route
-            if not cached:
-                ep.get_layout(idx[i], w.E, num_segments=w.S, expert_alignment=w.align,
-                              topk_weights=wts[i], handle=hs[i], recv_topk_idx=ri, recv_topk_weights=rw)
-            ep.dispatch_with_handle(xs[i], hs[i], use_fp8=True, recv_x=rq, recv_scales=rs)
+            if cached:
+                ep.dispatch_with_handle(xs[i], hs[i], use_fp8=True, recv_x=rq, recv_scales=rs)
+            else:   # layout + dispatch in one call (one kernel at this size)
+                ep.dispatch(xs[i], idx[i], wts[i], w.E, expert_alignment=w.align, num_segments=w.S,
+                            handle=hs[i], use_fp8=True, recv_x=rq, recv_scales=rs,
+                            recv_topk_idx=ri, recv_topk_weights=rw)
             ep.combine(y, hs[i], wts[i], out=out)
 
     result = {"config": "decode: T=128 hidden=7168 experts=256 topk=8 alignment=1 fp8 dispatch + "

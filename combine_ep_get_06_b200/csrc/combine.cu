@@ -5,7 +5,9 @@
 // fp32 FMA from +0 in ascending j, one bf16 rounding at the end.  A CTA
 // works on one unit = blockDim 16-byte column items (8 bf16) of one token:
 // each thread issues its (up to 8 per group) row loads before the FMAs, so
-// a thread keeps k 16-byte loads in flight.
+// a thread keeps k 16-byte loads in flight.  Launched with programmatic
+// dependent launch: the CTAs start while the previous grid finishes and
+// wait for it before reading anything.
 #include "ep_device.cuh"
 #include "ep_internal.h"
 
@@ -20,13 +22,15 @@ __global__ void __launch_bounds__(kMaxThreads) combine_kernel(CombineArgs a, int
     const int T = a.T, k = a.k, H = a.H;
     const char* const y = (const char*)a.y;
     const size_t row_bytes = (size_t)H * 2;
+    pdl_wait();
+    pdl_launch_dependents();
 
     // dispatch_backward's weight gradient: gather each slot's row value.
     if (a.out_weights != nullptr) {
         const int64_t n = (int64_t)T * k;
         for (int64_t i = (int64_t)blockIdx.x * blockDim.x + tid; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-            const int row = __ldg(a.slot_map + i);
-            a.out_weights[i] = (row >= 0 && row < a.max_rows) ? __ldg(a.recv_weights_in + row) : 0.0f;
+            const int row = ld_cg(a.slot_map + i);
+            a.out_weights[i] = (row >= 0 && row < a.max_rows) ? ld_cg(a.recv_weights_in + row) : 0.0f;
         }
     }
 
@@ -43,8 +47,8 @@ __global__ void __launch_bounds__(kMaxThreads) combine_kernel(CombineArgs a, int
             int row = -1;
             float wj = 1.0f;
             if (j < k) {
-                row = __ldg(a.slot_map + (size_t)t * k + j);
-                if (a.topk_weights != nullptr) wj = __ldg(a.topk_weights + (size_t)t * k + j);
+                row = a.slot_map[(size_t)t * k + j];
+                if (a.topk_weights != nullptr) wj = a.topk_weights[(size_t)t * k + j];
                 if (row >= a.max_rows) {
                     atomicOr(a.error_word, EP_DEVERR_CAPACITY);
                     row = -1;
@@ -109,8 +113,16 @@ cudaError_t launch_t(const CombineArgs& a, cudaStream_t stream) {
         if (gather > want) want = gather;
     }
     const int64_t grid = want < 1 ? 1 : (want < cap ? want : cap);
-    combine_kernel<G><<<(unsigned)grid, bd, 0, stream>>>(a, ipr, upr);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(bd);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, combine_kernel<G>, a, ipr, upr);
 }
 
 }  // namespace

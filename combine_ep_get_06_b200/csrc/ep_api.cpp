@@ -178,10 +178,14 @@ EP_API size_t ep_layout_workspace_bytes(const ep_handle* h) {
     return round256(C * h->num_experts * sizeof(int32_t)) + round256(C * h->num_segments * sizeof(int32_t));
 }
 
-EP_API ep_status ep_get_layout(ep_handle* h, const void* topk_idx, int32_t idx_is_int64,
-                               const float* topk_weights, int32_t* recv_topk_idx,
-                               float* recv_topk_weights, void* workspace, size_t workspace_bytes,
-                               ep_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Checks the layout arguments and fills a.
+ep_status prepare_layout(ep_handle* h, const void* topk_idx, int32_t idx_is_int64, const float* topk_weights,
+                         int32_t* recv_topk_idx, float* recv_topk_weights, void* workspace,
+                         size_t workspace_bytes, ep::LayoutArgs* a) {
     ep_status st = check_handle(h);
     if (st != EP_OK) return st;
     if (idx_is_int64 != 0 && idx_is_int64 != 1) return invalid("idx_is_int64 must be 0 or 1");
@@ -193,24 +197,21 @@ EP_API ep_status ep_get_layout(ep_handle* h, const void* topk_idx, int32_t idx_i
     const size_t need = ep_layout_workspace_bytes(h);
     if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need)
         return invalid("workspace must be 256-byte aligned with >= %zu bytes (got %zu)", need, workspace_bytes);
-
-    ep::LayoutArgs a;
-    a.topk_idx = topk_idx;
-    a.topk_weights = topk_weights;
-    a.recv_topk_idx = recv_topk_idx;
-    a.recv_topk_weights = recv_topk_weights;
-    a.h = *h;
-    a.chunk_tokens = ep::layout_chunk_tokens(h->num_topk);
-    a.num_chunks = ep::layout_num_chunks(h->num_tokens, h->num_topk);
-    a.ws_hist = (int32_t*)workspace;
-    a.ws_seg = (int32_t*)((char*)workspace + round256((size_t)a.num_chunks * h->num_experts * sizeof(int32_t)));
-    cudaError_t err = ep::launch_layout(a, idx_is_int64 == 1, (cudaStream_t)stream);
-    if (err != cudaSuccess) return cuda_failed("layout launch", err);
-    return ok();
+    a->topk_idx = topk_idx;
+    a->topk_weights = topk_weights;
+    a->recv_topk_idx = recv_topk_idx;
+    a->recv_topk_weights = recv_topk_weights;
+    a->h = *h;
+    a->chunk_tokens = ep::layout_chunk_tokens(h->num_topk);
+    a->num_chunks = ep::layout_num_chunks(h->num_tokens, h->num_topk);
+    a->ws_hist = (int32_t*)workspace;
+    a->ws_seg = (int32_t*)((char*)workspace + round256((size_t)a->num_chunks * h->num_experts * sizeof(int32_t)));
+    return EP_OK;
 }
 
-EP_API ep_status ep_dispatch(const ep_handle* h, ep_x_mode mode, const void* x, const float* x_scales,
-                             int32_t H, void* recv_x, float* recv_scales, ep_stream_t stream) {
+// Checks the dispatch arguments and fills a.
+ep_status prepare_dispatch(const ep_handle* h, ep_x_mode mode, const void* x, const float* x_scales, int32_t H,
+                           void* recv_x, float* recv_scales, ep::DispatchArgs* a) {
     ep_status st = check_handle(h);
     if (st != EP_OK) return st;
     if (mode != EP_X_BF16 && mode != EP_X_FP8 && mode != EP_X_BF16_TO_FP8) return invalid("unknown x mode %d", (int)mode);
@@ -223,21 +224,74 @@ EP_API ep_status ep_dispatch(const ep_handle* h, ep_x_mode mode, const void* x, 
         return invalid("recv_scales must be non-NULL and 4-byte aligned in the FP8 modes");
     if (mode == EP_X_FP8 && h->num_tokens > 0 && (x_scales == nullptr || !aligned(x_scales, 4)))
         return invalid("x_scales must be non-NULL and 4-byte aligned for pre-quantised x");
+    if (ep::dispatch_smem_bytes(mode, H) > ep::kMaxDispatchSmem)
+        return invalid("hidden %d is too large for this mode (row buffers exceed shared memory)", H);
+    a->x = x;
+    a->x_scales = x_scales;
+    a->recv_x = recv_x;
+    a->recv_scales = recv_scales;
+    a->slot_map = h->slot_map;
+    a->pad_rows = h->pad_rows;
+    a->num_pad_rows = h->num_pad_rows;
+    a->error_word = h->error_word;
+    a->T = h->num_tokens;
+    a->k = h->num_topk;
+    a->H = H;
+    a->max_rows = h->max_recv_rows;
+    a->max_pad_rows = h->num_experts * (h->expert_alignment - 1);
+    a->bulk_scales = fp8 && ((H / 128) * 4) % 16 == 0 && aligned(recv_scales, 16);
+    return EP_OK;
+}
 
+}  // namespace
+
+extern "C" {
+
+EP_API ep_status ep_get_layout(ep_handle* h, const void* topk_idx, int32_t idx_is_int64,
+                               const float* topk_weights, int32_t* recv_topk_idx,
+                               float* recv_topk_weights, void* workspace, size_t workspace_bytes,
+                               ep_stream_t stream) {
+    ep::LayoutArgs a;
+    ep_status st = prepare_layout(h, topk_idx, idx_is_int64, topk_weights, recv_topk_idx, recv_topk_weights,
+                                  workspace, workspace_bytes, &a);
+    if (st != EP_OK) return st;
+    cudaError_t err = ep::launch_layout(a, idx_is_int64 == 1, (cudaStream_t)stream);
+    if (err != cudaSuccess) return cuda_failed("layout launch", err);
+    return ok();
+}
+
+EP_API ep_status ep_dispatch(const ep_handle* h, ep_x_mode mode, const void* x, const float* x_scales,
+                             int32_t H, void* recv_x, float* recv_scales, ep_stream_t stream) {
     ep::DispatchArgs a;
-    a.x = x;
-    a.x_scales = x_scales;
-    a.recv_x = recv_x;
-    a.recv_scales = recv_scales;
-    a.slot_map = h->slot_map;
-    a.pad_rows = h->pad_rows;
-    a.num_pad_rows = h->num_pad_rows;
-    a.error_word = h->error_word;
-    a.T = h->num_tokens;
-    a.k = h->num_topk;
-    a.H = H;
-    a.max_rows = h->max_recv_rows;
+    ep_status st = prepare_dispatch(h, mode, x, x_scales, H, recv_x, recv_scales, &a);
+    if (st != EP_OK) return st;
     cudaError_t err = ep::launch_dispatch(a, mode, (cudaStream_t)stream);
+    if (err != cudaSuccess) return cuda_failed("dispatch launch", err);
+    return ok();
+}
+
+EP_API ep_status ep_layout_dispatch(ep_handle* h, const void* topk_idx, int32_t idx_is_int64,
+                                    const float* topk_weights, int32_t* recv_topk_idx,
+                                    float* recv_topk_weights, void* workspace, size_t workspace_bytes,
+                                    ep_x_mode mode, const void* x, const float* x_scales, int32_t H,
+                                    void* recv_x, float* recv_scales, ep_stream_t stream) {
+    ep::LayoutArgs la;
+    ep::DispatchArgs da;
+    ep_status st = prepare_layout(h, topk_idx, idx_is_int64, topk_weights, recv_topk_idx, recv_topk_weights,
+                                  workspace, workspace_bytes, &la);
+    if (st != EP_OK) return st;
+    st = prepare_dispatch(h, mode, x, x_scales, H, recv_x, recv_scales, &da);
+    if (st != EP_OK) return st;
+    cudaError_t err;
+    if (la.num_chunks == 1 &&
+        ep::layout_dispatch_smem_bytes(mode, H, h->num_experts, h->num_segments) <= ep::kMaxFusedSmem) {
+        err = ep::launch_layout_dispatch(la, da, mode, idx_is_int64 == 1, (cudaStream_t)stream);
+        if (err != cudaSuccess) return cuda_failed("fused layout+dispatch launch", err);
+        return ok();
+    }
+    err = ep::launch_layout(la, idx_is_int64 == 1, (cudaStream_t)stream);
+    if (err != cudaSuccess) return cuda_failed("layout launch", err);
+    err = ep::launch_dispatch(da, mode, (cudaStream_t)stream);
     if (err != cudaSuccess) return cuda_failed("dispatch launch", err);
     return ok();
 }

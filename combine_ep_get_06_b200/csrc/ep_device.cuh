@@ -1,5 +1,6 @@
 // Device helpers shared by the kernels: vector loads / stores with cache
-// hints and the bf16 / e4m3 conversions.
+// hints, bf16 / e4m3 conversions, TMA bulk copies and programmatic
+// dependent launch.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -9,22 +10,27 @@
 
 namespace ep {
 
-// 16-byte read-only load that does not allocate in L1 (every byte of the
-// streamed inputs is read once).
+// 16-byte load of streamed data that does not allocate in L1 (every byte
+// is read once).  Not the non-coherent path: with programmatic dependent
+// launch the data may come from the grid that ran just before.
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
     uint4 v;
-    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-        : "l"(p));
+    asm volatile("ld.global.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
     return v;
 }
 
-// 16-byte store of output that is not read again by this kernel.
+// 16-byte store of output that this kernel does not read again.
 __device__ __forceinline__ void st_stream(void* p, const uint4& v) {
     asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
                  "r"(v.w)
                  : "memory");
 }
+
+// Coherent (L2) scalar loads, for data the previous grid may have written.
+__device__ __forceinline__ int ld_cg(const int* p) { return __ldcg(p); }
+__device__ __forceinline__ float ld_cg(const float* p) { return __ldcg(p); }
 
 // Two packed bf16 (low half first) -> two floats, exactly.
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
@@ -47,5 +53,42 @@ __device__ __forceinline__ unsigned lanemask_lt() {
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
     return m;
 }
+
+// ---- programmatic dependent launch (no-ops when launched without it)
+
+// Blocks until the grids this one depends on have completed and their
+// memory is visible.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next grid in the stream begin launching.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---- TMA bulk copies shared -> global (never multicast)
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Makes this thread's generic-proxy shared-memory writes visible to the
+// async proxy (the TMA engine) before a bulk copy reads them.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// bytes: multiple of 16; both addresses 16-byte aligned.
+__device__ __forceinline__ void bulk_s2g(void* gdst, const void* ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+                 "r"(smem_addr(ssrc)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until at most N committed groups of this thread still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Waits until all committed groups of this thread have completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 }  // namespace ep

@@ -9,10 +9,10 @@
 
 namespace ep {
 
-// Layout: slots are processed in chunks of whole tokens, about
-// kLayoutChunkSlots slots each, one CTA per chunk.
+// Layout: one thread per slot; slots are processed in chunks of whole
+// tokens of at most kLayoutChunkSlots slots, one CTA per chunk.
 constexpr int kLayoutThreads = 1024;
-constexpr int kLayoutChunkSlots = 2048;
+constexpr int kLayoutChunkSlots = kLayoutThreads;
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopk = 32;
 
@@ -47,9 +47,21 @@ struct DispatchArgs {
     const int32_t* num_pad_rows;
     uint32_t* error_word;
     int32_t T, k, H, max_rows;
+    int32_t max_pad_rows;  // E*(alignment-1): bound on the padding rows
+    int32_t bulk_scales;  // scale rows are a multiple of 16 bytes and recv_scales is 16-byte aligned
 };
 
+// Shared memory one dispatch CTA needs for this mode and hidden size.
+size_t dispatch_smem_bytes(ep_x_mode mode, int H);
+constexpr size_t kMaxDispatchSmem = 200 * 1024;
+
 cudaError_t launch_dispatch(const DispatchArgs& a, ep_x_mode mode, cudaStream_t stream);
+
+// Fused layout + dispatch for T*k <= kLayoutThreads.
+size_t layout_dispatch_smem_bytes(ep_x_mode mode, int H, int E, int S);
+constexpr size_t kMaxFusedSmem = 220 * 1024;
+cudaError_t launch_layout_dispatch(const LayoutArgs& a, const DispatchArgs& d, ep_x_mode mode,
+                                   bool idx_is_int64, cudaStream_t stream);
 
 struct CombineArgs {
     const void* y;

@@ -1,0 +1,229 @@
+// Fused layout + dispatch for small batches (T*k <= 1024 slots, e.g. the
+// decode step): the dispatch(x, topk_idx, topk_weights, ...) call of the
+// DeepEP V2 README ("Interfaces and examples") in one launch.
+//
+// Every CTA (1024 threads, one per slot) computes the whole small layout in
+// shared memory -- the same steps as the single-CTA layout kernel -- so no
+// CTA waits for another.  CTA c then owns the tokens t = c, c+G, ...: it
+// writes their slot-map entries and per-row arrays, quantises or copies
+// their x rows into a shared row buffer and bulk-copies (TMA, no multicast)
+// that buffer to the k receive rows; it also writes its share of the
+// padding rows.  Each CTA loads the x row of its first token before the
+// layout, so that load overlaps the layout's latency.
+#include "layout_device.cuh"
+
+namespace ep {
+namespace {
+
+using namespace layout_dev;
+
+constexpr float kE4m3Max = 448.0f;
+constexpr float kAmaxFloor = 1e-4f;
+
+struct FusedGeometry {
+    int row_bytes, ipr, scale_bytes, scale_pad;
+    size_t layout_off, row_off, scale_off, zero_off, srow_off, total;
+};
+
+__host__ __device__ inline FusedGeometry fused_geometry(int mode, int H, int E, int S) {
+    FusedGeometry g;
+    const bool fp8 = mode != EP_X_BF16;
+    g.row_bytes = fp8 ? H : 2 * H;
+    g.ipr = g.row_bytes / 16;
+    g.scale_bytes = fp8 ? (H / 128) * 4 : 0;
+    g.scale_pad = (g.scale_bytes + 15) & ~15;
+    g.layout_off = 0;
+    g.row_off = (layout_dev::smem_bytes(E, S) + 127) & ~(size_t)127;
+    g.scale_off = g.row_off + g.row_bytes;
+    g.zero_off = g.scale_off + g.scale_pad;
+    g.srow_off = g.zero_off + g.row_bytes + g.scale_pad;
+    g.total = g.srow_off + sizeof(int) * kThreads;
+    return g;
+}
+
+// Quantises (or copies) item c of token t's row into the row buffer.
+template <int kMode>
+__device__ __forceinline__ void fill_item(const DispatchArgs& d, int t, int c, bool active, uint4 v0, uint4 v1,
+                                          unsigned char* rb, float* sb) {
+    if (kMode == EP_X_BF16_TO_FP8) {
+        float f[16] = {bf16_lo(v0.x), bf16_hi(v0.x), bf16_lo(v0.y), bf16_hi(v0.y),
+                       bf16_lo(v0.z), bf16_hi(v0.z), bf16_lo(v0.w), bf16_hi(v0.w),
+                       bf16_lo(v1.x), bf16_hi(v1.x), bf16_lo(v1.y), bf16_hi(v1.y),
+                       bf16_lo(v1.z), bf16_hi(v1.z), bf16_lo(v1.w), bf16_hi(v1.w)};
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+        amax = fmaxf(amax, kAmaxFloor);
+        const float scale = __fdiv_rn(amax, kE4m3Max);
+        const float inv = __fdiv_rn(kE4m3Max, amax);
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            w[i] = pack_e4m3x2(__fmul_rn(f[4 * i], inv), __fmul_rn(f[4 * i + 1], inv)) |
+                   (pack_e4m3x2(__fmul_rn(f[4 * i + 2], inv), __fmul_rn(f[4 * i + 3], inv)) << 16);
+        if (active) {
+            reinterpret_cast<uint4*>(rb)[c] = make_uint4(w[0], w[1], w[2], w[3]);
+            if ((c & 7) == 0) sb[c >> 3] = scale;
+        }
+    } else if (active) {
+        reinterpret_cast<uint4*>(rb)[c] = v0;
+        if (kMode == EP_X_FP8 && (c & 7) == 0) sb[c >> 3] = __ldg(d.x_scales + (size_t)t * (d.H / 128) + (c >> 3));
+    }
+}
+
+template <int kMode>
+__device__ __forceinline__ void load_item(const DispatchArgs& d, int t, int c, bool active, uint4& v0, uint4& v1) {
+    v0 = v1 = make_uint4(0, 0, 0, 0);
+    if (!active) return;
+    if (kMode == EP_X_BF16_TO_FP8) {
+        const char* src = (const char*)d.x + (size_t)t * d.H * 2 + (size_t)c * 32;
+        v0 = ld_stream(src);
+        v1 = ld_stream(src + 16);
+    } else {
+        const size_t rb = kMode == EP_X_BF16 ? (size_t)d.H * 2 : (size_t)d.H;
+        v0 = ld_stream((const char*)d.x + (size_t)t * rb + (size_t)c * 16);
+    }
+}
+
+template <typename IdxT, int kMode>
+__global__ void __launch_bounds__(kThreads) layout_dispatch_kernel(LayoutArgs a, DispatchArgs d) {
+    constexpr bool kFp8Out = kMode != EP_X_BF16;
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int E = a.h.num_experts, S = a.h.num_segments, k = a.h.num_topk, T = a.h.num_tokens;
+    const FusedGeometry geo = fused_geometry(kMode, d.H, E, S);
+    Smem m(reinterpret_cast<int*>(smem + geo.layout_off), E, S);
+    unsigned char* rb = smem + geo.row_off;
+    float* sb = reinterpret_cast<float*>(smem + geo.scale_off);
+    unsigned char* zeros = smem + geo.zero_off;
+    int* srow = reinterpret_cast<int*>(smem + geo.srow_off);  // [kThreads] row of each slot
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int c_cta = blockIdx.x, G = gridDim.x;
+    const int64_t s = tid;
+    const bool has_slot = s < (int64_t)T * k;
+    char* const recv = (char*)d.recv_x;
+    char* const rscl = (char*)d.recv_scales;
+
+    // Loads first: this thread's slot, and its item of the first token row.
+    bool bad = false;
+    int e = -1;
+    float wv = 0.0f;
+    if (has_slot) {
+        e = read_expert((const IdxT*)a.topk_idx, s, E, bad);
+        if (a.topk_weights) wv = __ldg(a.topk_weights + s);
+    }
+    uint4 pre0, pre1;
+    const bool first_active = c_cta < T && tid < geo.ipr;
+    load_item<kMode>(d, c_cta, tid, first_active, pre0, pre1);
+    for (int i = tid; i < (geo.row_bytes + geo.scale_pad) / 16; i += kThreads)
+        reinterpret_cast<uint4*>(zeros)[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+
+    const SlotRank r = small_layout<IdxT>(a, m, e, bad);
+    const int row_s = slot_row(m, r, E);
+    srow[tid] = (row_s < a.h.max_recv_rows) ? row_s : -1;
+    if (has_slot && (int)(s / k) % G == c_cta) write_slot(a, s, row_s, e, wv);
+    if (c_cta == 0) {
+        write_totals(a, m, E);
+        for (int g = tid; g < S; g += blockDim.x) a.h.seg_tokens[g] = m.seg[g];
+    }
+    const int P = m.padoff[E];
+    const int p0 = (int)((int64_t)P * c_cta / G), p1 = (int)((int64_t)P * (c_cta + 1) / G);
+    write_padding(a, m, E, p0, p1);
+    pdl_launch_dependents();
+    __syncthreads();
+
+    // Padding rows of this CTA's share: bulk copies of zeros.
+    if (warp == 0) {
+        for (int p = p0 + lane; p < p1; p += 32) {
+            const int row = pad_row(m, E, p);
+            if (row >= a.h.max_recv_rows) continue;
+            bulk_s2g(recv + (size_t)row * geo.row_bytes, zeros, geo.row_bytes);
+            if (d.bulk_scales) bulk_s2g(rscl + (size_t)row * geo.scale_bytes, zeros + geo.row_bytes, geo.scale_bytes);
+            bulk_commit();
+            if (kFp8Out && !d.bulk_scales)
+                for (int b = 0; b < d.H / 128; ++b) d.recv_scales[(size_t)row * (d.H / 128) + b] = 0.0f;
+        }
+    }
+
+    bool first = true;
+    for (int t = c_cta; t < T; t += G) {
+        if (!first) {
+            if (warp == 0) bulk_wait_read<0>();
+            __syncthreads();
+        }
+        for (int c0 = warp * 32; c0 < geo.ipr; c0 += kThreads) {
+            const int c = c0 + lane;
+            const bool active = c < geo.ipr;
+            uint4 v0, v1;
+            if (first && c0 == warp * 32) {
+                v0 = pre0;
+                v1 = pre1;
+            } else {
+                load_item<kMode>(d, t, c, active, v0, v1);
+            }
+            fill_item<kMode>(d, t, c, active, v0, v1, rb, sb);
+        }
+        first = false;
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (warp == 0 && lane < k) {
+            const int row = srow[t * k + lane];
+            if (row >= 0) {
+                bulk_s2g(recv + (size_t)row * geo.row_bytes, rb, geo.row_bytes);
+                if (d.bulk_scales) bulk_s2g(rscl + (size_t)row * geo.scale_bytes, sb, geo.scale_bytes);
+            }
+            bulk_commit();
+        }
+        if (kFp8Out && !d.bulk_scales) {
+            const int B = d.H / 128;
+            for (int i = tid; i < k * B; i += kThreads) {
+                const int row = srow[t * k + i / B];
+                if (row >= 0) d.recv_scales[(size_t)row * B + i % B] = sb[i % B];
+            }
+        }
+    }
+    if (warp == 0) bulk_wait_all();
+}
+
+template <typename IdxT, int kMode>
+cudaError_t launch_t(const LayoutArgs& a, const DispatchArgs& d, cudaStream_t stream) {
+    const FusedGeometry g = fused_geometry(kMode, d.H, a.h.num_experts, a.h.num_segments);
+    auto kernel = layout_dispatch_kernel<IdxT, kMode>;
+    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.total);
+    if (err != cudaSuccess) return err;
+    int grid = a.h.num_tokens < device_sm_count() ? a.h.num_tokens : device_sm_count();
+    if (grid < 1) grid = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = g.total;
+    cfg.stream = stream;
+    return cudaLaunchKernelEx(&cfg, kernel, a, d);
+}
+
+template <typename IdxT>
+cudaError_t launch_mode(const LayoutArgs& a, const DispatchArgs& d, ep_x_mode mode, cudaStream_t stream) {
+    switch (mode) {
+        case EP_X_BF16: return launch_t<IdxT, EP_X_BF16>(a, d, stream);
+        case EP_X_FP8: return launch_t<IdxT, EP_X_FP8>(a, d, stream);
+        case EP_X_BF16_TO_FP8: return launch_t<IdxT, EP_X_BF16_TO_FP8>(a, d, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+size_t layout_dispatch_smem_bytes(ep_x_mode mode, int H, int E, int S) {
+    return fused_geometry(mode, H, E, S).total;
+}
+
+cudaError_t launch_layout_dispatch(const LayoutArgs& a, const DispatchArgs& d, ep_x_mode mode, bool idx_is_int64,
+                                   cudaStream_t stream) {
+    return idx_is_int64 ? launch_mode<long long>(a, d, mode, stream) : launch_mode<int>(a, d, mode, stream);
+}
+
+}  // namespace ep

@@ -57,6 +57,8 @@ SIGNATURES = {
     "ep_layout_workspace_bytes": (_SZ, [_HP]),
     "ep_get_layout": (ctypes.c_int, [_HP, _P, _I32, _P, _P, _P, _P, _SZ, _P]),
     "ep_dispatch": (ctypes.c_int, [_HP, ctypes.c_int, _P, _P, _I32, _P, _P, _P]),
+    "ep_layout_dispatch": (ctypes.c_int, [_HP, _P, _I32, _P, _P, _P, _P, _SZ, ctypes.c_int, _P, _P, _I32,
+                                          _P, _P, _P]),
     "ep_combine": (ctypes.c_int, [_HP, _P, _I32, _P, _P, _P, _P, _P]),
     "ep_read_total_rows": (ctypes.c_int, [_HP, ctypes.POINTER(_I32), _P]),
     "ep_check_error": (ctypes.c_int, [_HP, ctypes.POINTER(ctypes.c_uint32), _P]),
@@ -239,13 +241,9 @@ def get_layout(topk_idx: torch.Tensor, num_experts: int, *, num_segments: int = 
 XType = Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]]
 
 
-def dispatch_with_handle(x: XType, handle: EPHandle, *, use_fp8: bool = False,
-                         recv_x: Optional[torch.Tensor] = None,
-                         recv_scales: Optional[torch.Tensor] = None):
-    """Dispatch with an existing handle (decode with a cached handle; the
-    backward of combine).  x bf16 [T,H] -> recv_x bf16 [max_recv_rows,H];
-    x bf16 with use_fp8 -> (recv_x e4m3 [rows,H], recv_scales f32 [rows,H/128]);
-    x = (x_fp8 [T,H], scales [T,H/128]) -> the same tuple, copied."""
+def _dispatch_args(x: XType, handle: EPHandle, use_fp8: bool, recv_x, recv_scales):
+    """Checks x and the receive buffers (allocating those not given);
+    returns (mode, x, x_scales, H, recv_x, recv_scales)."""
     dev = handle.device
     rows = handle.max_recv_rows
     x_scales = None
@@ -260,6 +258,8 @@ def dispatch_with_handle(x: XType, handle: EPHandle, *, use_fp8: bool = False,
     T, H = x.shape
     if T != handle.num_tokens:
         raise ValueError(f"x has {T} rows, handle has {handle.num_tokens} tokens")
+    if mode == EP_X_FP8 and tuple(x_scales.shape) != (T, H // 128):
+        raise ValueError("x scales must be [T, hidden/128]")
     if mode == EP_X_BF16:
         if recv_x is None:
             recv_x = torch.empty(rows, H, dtype=torch.bfloat16, device=dev)
@@ -275,29 +275,64 @@ def dispatch_with_handle(x: XType, handle: EPHandle, *, use_fp8: bool = False,
             raise ValueError("recv_scales must be [max_recv_rows, hidden/128]")
     if tuple(recv_x.shape) != (rows, H):
         raise ValueError("recv_x must be [max_recv_rows, hidden]")
+    return mode, x, x_scales, H, recv_x, recv_scales
+
+
+def dispatch_with_handle(x: XType, handle: EPHandle, *, use_fp8: bool = False,
+                         recv_x: Optional[torch.Tensor] = None,
+                         recv_scales: Optional[torch.Tensor] = None):
+    """Dispatch with an existing handle (decode with a cached handle; the
+    backward of combine).  x bf16 [T,H] -> recv_x bf16 [max_recv_rows,H];
+    x bf16 with use_fp8 -> (recv_x e4m3 [rows,H], recv_scales f32 [rows,H/128]);
+    x = (x_fp8 [T,H], scales [T,H/128]) -> the same tuple, copied."""
+    mode, x, x_scales, H, recv_x, recv_scales = _dispatch_args(x, handle, use_fp8, recv_x, recv_scales)
     _check(lib().ep_dispatch(handle.ref, mode, x.data_ptr(), _ptr(x_scales), H, recv_x.data_ptr(),
-                             _ptr(recv_scales), _stream(dev)), "dispatch")
+                             _ptr(recv_scales), _stream(handle.device)), "dispatch")
     return recv_x if mode == EP_X_BF16 else (recv_x, recv_scales)
 
 
 def dispatch(x: XType, topk_idx: Optional[torch.Tensor] = None,
              topk_weights: Optional[torch.Tensor] = None, num_experts: Optional[int] = None, *,
              expert_alignment: int = 1, num_segments: int = 1, handle: Optional[EPHandle] = None,
-             use_fp8: bool = False, max_recv_rows: Optional[int] = None):
-    """MoE dispatch.  With topk_idx: computes the layout, then dispatches;
-    returns (recv_x, recv_topk_idx, recv_topk_weights, handle).  With only a
-    handle (cached): returns (recv_x, None, None, handle)."""
+             use_fp8: bool = False, max_recv_rows: Optional[int] = None,
+             recv_x: Optional[torch.Tensor] = None, recv_scales: Optional[torch.Tensor] = None,
+             recv_topk_idx: Optional[torch.Tensor] = None,
+             recv_topk_weights: Optional[torch.Tensor] = None):
+    """MoE dispatch.  With topk_idx: layout and dispatch in one call (one
+    kernel for small batches); returns (recv_x, recv_topk_idx,
+    recv_topk_weights, handle).  With only a handle (cached): returns
+    (recv_x, None, None, handle)."""
     if topk_idx is None:
         if handle is None:
             raise ValueError("dispatch needs topk_idx or a handle")
-        return dispatch_with_handle(x, handle, use_fp8=use_fp8), None, None, handle
+        return dispatch_with_handle(x, handle, use_fp8=use_fp8, recv_x=recv_x,
+                                    recv_scales=recv_scales), None, None, handle
     if num_experts is None:
         raise ValueError("num_experts is required with topk_idx")
-    handle, recv_idx, recv_w = get_layout(topk_idx, num_experts, num_segments=num_segments,
-                                          expert_alignment=expert_alignment,
-                                          topk_weights=topk_weights, handle=handle,
-                                          max_recv_rows=max_recv_rows)
-    return dispatch_with_handle(x, handle, use_fp8=use_fp8), recv_idx, recv_w, handle
+    _need(topk_idx, "topk_idx", (torch.int64, torch.int32), ndim=2)
+    T, k = topk_idx.shape
+    dev = topk_idx.device
+    if handle is None:
+        handle = EPHandle(T, k, num_experts, num_segments, expert_alignment, max_recv_rows, device=dev)
+    elif (handle.num_tokens, handle.num_topk, handle.num_experts) != (T, k, num_experts):
+        raise ValueError("handle shape does not match topk_idx / num_experts")
+    if topk_weights is not None:
+        _need(topk_weights, "topk_weights", (torch.float32,), dev, 2)
+        if tuple(topk_weights.shape) != (T, k):
+            raise ValueError("topk_weights must have the shape of topk_idx")
+    R = handle.max_recv_rows
+    ri = torch.empty(R, dtype=torch.int32, device=dev) if recv_topk_idx is None else recv_topk_idx
+    rw = torch.empty(R, dtype=torch.float32, device=dev) if recv_topk_weights is None else recv_topk_weights
+    _need(ri, "recv_topk_idx", (torch.int32,), dev, 1)
+    _need(rw, "recv_topk_weights", (torch.float32,), dev, 1)
+    mode, x, x_scales, H, recv_x, recv_scales = _dispatch_args(x, handle, use_fp8, recv_x, recv_scales)
+    _check(lib().ep_layout_dispatch(handle.ref, topk_idx.data_ptr(), int(topk_idx.dtype == torch.int64),
+                                    _ptr(topk_weights), ri.data_ptr(), rw.data_ptr(),
+                                    handle.workspace_ptr, handle.workspace_bytes, mode, x.data_ptr(),
+                                    _ptr(x_scales), H, recv_x.data_ptr(), _ptr(recv_scales),
+                                    _stream(dev)), "dispatch")
+    out = recv_x if mode == EP_X_BF16 else (recv_x, recv_scales)
+    return out, ri, rw, handle
 
 
 def combine(y: torch.Tensor, handle: EPHandle, topk_weights: Optional[torch.Tensor] = None, *,

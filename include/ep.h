@@ -165,6 +165,20 @@ EP_API ep_status ep_dispatch(const ep_handle* handle, ep_x_mode mode, const void
                              const float* x_scales, int32_t hidden, void* recv_x,
                              float* recv_scales, ep_stream_t stream);
 
+/* Layout and dispatch in one call: the dispatch(x, topk_idx, topk_weights,
+ * num_experts, expert_alignment) call of the DeepEP V2 README ("Interfaces
+ * and examples"), which routes and sends in one step.  Arguments, results
+ * and errors are those of ep_get_layout followed by ep_dispatch with the
+ * same handle.  When T*k <= 1024 (a decode step) it runs as ONE kernel in
+ * which every CTA computes the small layout itself, instead of two or
+ * three launches; otherwise it launches the same kernels as the two calls. */
+EP_API ep_status ep_layout_dispatch(ep_handle* handle, const void* topk_idx, int32_t idx_is_int64,
+                                    const float* topk_weights, int32_t* recv_topk_idx,
+                                    float* recv_topk_weights, void* workspace,
+                                    size_t workspace_bytes, ep_x_mode mode, const void* x,
+                                    const float* x_scales, int32_t hidden, void* recv_x,
+                                    float* recv_scales, ep_stream_t stream);
+
 /* Combine (combine_forward; unweighted it is dispatch_backward):
  *   out[t,:] = bf16( sum_j w[t,j] * y[slot_map[t*k+j],:] ) over valid slots,
  *   accumulated in fp32 as acc = fma(w, y, acc) from +0 in ascending j and

@@ -153,3 +153,46 @@ def max_bf16_ulp_diff(a_bits: np.ndarray, b_bits: np.ndarray) -> int:
         b = b.astype(np.int32)
         return np.where(b & 0x8000, 0x8000 - (b & 0x7FFF), 0x8000 + (b & 0x7FFF))
     return int(np.abs(ordered(a_bits) - ordered(b_bits)).max(initial=0))
+
+
+def run_cuda_fused(inp: dict, w: W.Workload, mode: int, *, prequant=None):
+    """layout + dispatch through ep.dispatch(x, topk_idx, ...) (one kernel
+    when T*k <= 1024); returns host arrays like run_cuda (no combine)."""
+    T = inp["x"].shape[0]
+    idx = torch.from_numpy(inp["topk_idx"]).cuda()
+    wts = torch.from_numpy(inp["topk_weights"]).cuda()
+    handle = ep.EPHandle(T, w.k, w.E, w.S, w.align, device="cuda")
+    rows = handle.max_recv_rows
+    ri_buf, recv_idx = guarded(rows, 1, torch.int32)
+    rw_buf, recv_w = guarded(rows, 1, torch.float32)
+    H = w.H
+    out = {"handle": handle}
+    if mode == ep.EP_X_BF16:
+        rx_buf, recv_x = guarded(rows, H, torch.bfloat16)
+        ep.dispatch(to_dev_bf16(inp["x"]), idx, wts, w.E, expert_alignment=w.align, num_segments=w.S,
+                    handle=handle, recv_x=recv_x, recv_topk_idx=recv_idx.view(-1),
+                    recv_topk_weights=recv_w.view(-1))
+        out["recv_x"] = bits16(recv_x)
+        out["guards"] = [(rx_buf, rows * H * 2)]
+    else:
+        rx_buf, recv_x = guarded(rows, H, torch.uint8)
+        rs_buf, recv_s = guarded(rows, H // 128, torch.float32)
+        if mode == ep.EP_X_FP8:
+            xin = (torch.from_numpy(prequant[0]).cuda(), torch.from_numpy(prequant[1]).cuda())
+        else:
+            xin = to_dev_bf16(inp["x"])
+        ep.dispatch(xin, idx, wts, w.E, expert_alignment=w.align, num_segments=w.S, handle=handle,
+                    use_fp8=True, recv_x=recv_x, recv_scales=recv_s, recv_topk_idx=recv_idx.view(-1),
+                    recv_topk_weights=recv_w.view(-1))
+        out["recv_x"] = bytes8(recv_x)
+        out["recv_scales"] = recv_s.cpu().numpy()
+        out["guards"] = [(rx_buf, rows * H), (rs_buf, rows * (H // 128) * 4)]
+    out["guards"] += [(ri_buf, rows * 4), (rw_buf, rows * 4)]
+    torch.cuda.synchronize()
+    out["recv_topk_idx"] = recv_idx.view(-1).cpu().numpy()
+    out["recv_topk_weights"] = recv_w.view(-1).cpu().numpy()
+    for key in ("counts", "num_recv_tokens_per_expert", "offsets", "seg_tokens", "slot_map",
+                "recv_src", "pad_rows", "num_pad_rows"):
+        out[key] = getattr(handle, key).cpu().numpy()
+    out["error_bits"] = handle.check_error() if not _has_bad_idx(inp, w) else None
+    return out
