@@ -7,7 +7,8 @@
 // each thread issues its (up to 8 per group) row loads before the FMAs, so
 // a thread keeps k 16-byte loads in flight.  Launched with programmatic
 // dependent launch: the CTAs start while the previous grid finishes and
-// wait for it before reading anything.
+// wait for it before reading anything; each lets the next grid start
+// launching once its own work is issued.
 #include "ep_device.cuh"
 #include "ep_internal.h"
 
@@ -23,7 +24,6 @@ __global__ void __launch_bounds__(kMaxThreads) combine_kernel(CombineArgs a, int
     const char* const y = (const char*)a.y;
     const size_t row_bytes = (size_t)H * 2;
     pdl_wait();
-    pdl_launch_dependents();
 
     // dispatch_backward's weight gradient: gather each slot's row value.
     if (a.out_weights != nullptr) {
@@ -88,6 +88,7 @@ __global__ void __launch_bounds__(kMaxThreads) combine_kernel(CombineArgs a, int
                                    pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
         st_stream((char*)a.out + (size_t)t * row_bytes + (size_t)c * 16, o);
     }
+    pdl_launch_dependents();
 }
 
 int unit_threads(int ipr) {

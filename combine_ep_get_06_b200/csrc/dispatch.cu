@@ -8,7 +8,9 @@
 // a handful of copy instructions per row instead of k stores per 16 bytes.
 // Two row buffers alternate, so quantising row i+1 overlaps the copies of
 // row i.  Padding rows are written by bulk copies of a zeroed buffer, one
-// row per lane of warp 0.
+// row per lane of warp 0.  Launched with programmatic dependent launch: a
+// CTA waits for the previous grid before reading anything, and lets the
+// next grid start launching once it has issued all its copies.
 //
 // A CTA walks rows grid-stride: token rows [0, T), then padding batches of
 // 32 rows.  In the quantising mode a 1x128 block is 8 consecutive lanes
@@ -68,7 +70,6 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchArgs a) {
 
     // Everything below may read what the layout (the previous grid) wrote.
     pdl_wait();
-    pdl_launch_dependents();
     const int n_pad = ld_cg(a.num_pad_rows);
     const int n_pad_batches = (n_pad + 31) / 32;
     __syncthreads();
@@ -164,6 +165,8 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchArgs a) {
             }
         }
     }
+    // Let the next grid start launching while the copies drain.
+    pdl_launch_dependents();
     if (warp == 0) bulk_wait_all();
 }
 

@@ -22,11 +22,10 @@ using namespace layout_dev;
 
 template <typename IdxT>
 __global__ void __launch_bounds__(kThreads) layout_single_kernel(LayoutArgs a) {
-    extern __shared__ int smem_raw[];
+    extern __shared__ __align__(16) int smem_raw[];
     const int E = a.h.num_experts, S = a.h.num_segments;
     Smem m(smem_raw, E, S);
-    const int tid = threadIdx.x;
-    const int64_t s = tid;
+    const int64_t s = threadIdx.x;
     const bool has_slot = s < (int64_t)a.h.num_tokens * a.h.num_topk;
     bool bad = false;
     int e = -1;
@@ -36,19 +35,20 @@ __global__ void __launch_bounds__(kThreads) layout_single_kernel(LayoutArgs a) {
         if (a.topk_weights) wv = __ldg(a.topk_weights + s);
     }
     pdl_launch_dependents();
-    const SlotRank r = small_layout<IdxT>(a, m, e, bad);
-    if (has_slot) write_slot(a, s, slot_row(m, r, E), e, wv);
-    write_totals(a, m, E);
-    for (int g = tid; g < S; g += blockDim.x) a.h.seg_tokens[g] = m.seg[g];
+    const int row = small_layout<IdxT>(a, m, e, bad, wv);
+    if (has_slot) a.h.slot_map[s] = row;
+    write_rows(a, m, 0, m.lcoff[E]);
+    write_totals(a, m, E, S);
     write_padding(a, m, E, 0, m.padoff[E]);
 }
 
 template <typename IdxT>
 __global__ void __launch_bounds__(kThreads) layout_count_kernel(LayoutArgs a) {
-    extern __shared__ int smem_raw[];
+    extern __shared__ __align__(16) int smem_raw[];
     const int E = a.h.num_experts, S = a.h.num_segments, k = a.h.num_topk;
     int* hist = smem_raw;
     int* seg = smem_raw + E;
+    unsigned* tmask = reinterpret_cast<unsigned*>(seg + S);  // [2*kThreads]
     const int c = blockIdx.x, tid = threadIdx.x;
     const int t0 = c * a.chunk_tokens;
     const int t1 = min(a.h.num_tokens, t0 + a.chunk_tokens);
@@ -60,19 +60,25 @@ __global__ void __launch_bounds__(kThreads) layout_count_kernel(LayoutArgs a) {
     if (s < (int64_t)t1 * k) e = read_expert(idx, s, E, bad);
     pdl_launch_dependents();
     for (int i = tid; i < E + S; i += blockDim.x) smem_raw[i] = 0;
+    tmask[2 * tid] = 0;
+    tmask[2 * tid + 1] = 0;
     if (bad) atomicOr(a.h.error_word, EP_DEVERR_BAD_TOPK_IDX);
     __syncthreads();
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    if (e >= 0 && (peers & lanemask_lt()) == 0) atomicAdd(&hist[e], __popc(peers));
-    count_segments(idx, t0, t1, k, E, S, e, seg);
+    if (e >= 0) atomicAdd(&hist[e], 1);
+    if (S <= 64) mark_segment(tmask, tid / k, e, E, S);
+    else count_segments_walk(idx, t0, t1, k, E, S, seg);
     __syncthreads();
+    if (S <= 64) {
+        count_segments_masks(tmask, t1 - t0, S, seg);
+        __syncthreads();
+    }
     for (int i = tid; i < E; i += blockDim.x) a.ws_hist[(int64_t)c * E + i] = hist[i];
     for (int i = tid; i < S; i += blockDim.x) a.ws_seg[(int64_t)c * S + i] = seg[i];
 }
 
 template <typename IdxT>
 __global__ void __launch_bounds__(kThreads) layout_assign_kernel(LayoutArgs a) {
-    extern __shared__ int smem_raw[];
+    extern __shared__ __align__(16) int smem_raw[];
     const int E = a.h.num_experts, S = a.h.num_segments, k = a.h.num_topk;
     Smem m(smem_raw, E, S);
     const int c = blockIdx.x, C = gridDim.x, tid = threadIdx.x;
@@ -89,16 +95,18 @@ __global__ void __launch_bounds__(kThreads) layout_assign_kernel(LayoutArgs a) {
         e = read_expert((const IdxT*)a.topk_idx, s, E, ignore);
         if (a.topk_weights) wv = __ldg(a.topk_weights + s);
     }
-    for (int i = tid; i < kWarps * E; i += blockDim.x) m.tab[i] = 0;
+    zero_tab(m.tab, E);
     for (int i = tid; i < E; i += blockDim.x) {
         m.cnt[i] = 0;
         m.base[i] = 0;
     }
     for (int i = tid; i < S; i += blockDim.x) m.seg[i] = 0;
     __syncthreads();
-    const SlotRank r = rank_in_warp(e, m.tab, E);
+    mark_slot(e, m.tab, E);
     __syncthreads();
-    if (tid < E) column_scan(m.tab, E);
+    const int wrank = rank_in_warp(e, m.tab, E);
+    __syncthreads();
+    if (tid < E) m.lc[tid] = column_scan(m.tab, E);
 
     // Histograms of every chunk: totals, and the part from earlier chunks.
     pdl_wait();
@@ -106,15 +114,17 @@ __global__ void __launch_bounds__(kThreads) layout_assign_kernel(LayoutArgs a) {
     reduce_columns(a.ws_hist, a.num_chunks, E, c, m.cnt, m.base);
     if (c == 0) reduce_columns(a.ws_seg, a.num_chunks, S, 0, m.seg, nullptr);
     __syncthreads();
-    aligned_offsets(m, E, a.h.expert_alignment);
+    expert_offsets(m, E, a.h.expert_alignment);
     if (tid < E) m.base[tid] += m.off[tid];
     __syncthreads();
 
-    if (has_slot) write_slot(a, s, slot_row(m, r, E), e, wv);
-    if (c == 0) {
-        write_totals(a, m, E);
-        for (int g = tid; g < S; g += blockDim.x) a.h.seg_tokens[g] = m.seg[g];
-    }
+    const int crank = chunk_rank(m, e, wrank, E);
+    stage_slot(m, s, e, crank, wv);
+    const int row = slot_row(a, m, e, crank);
+    if (has_slot) a.h.slot_map[s] = row;
+    __syncthreads();
+    write_rows(a, m, 0, m.lcoff[E]);
+    if (c == 0) write_totals(a, m, E, S);
     const int P = m.padoff[E];
     write_padding(a, m, E, (int)((int64_t)P * c / C), (int)((int64_t)P * (c + 1) / C));
 }
@@ -148,7 +158,8 @@ cudaError_t launch_layout_t(const LayoutArgs& a, cudaStream_t stream) {
             return err;
     }
     if (a.num_chunks == 1) return launch(single, 1, smem, stream, false, a);
-    err = launch(layout_count_kernel<IdxT>, a.num_chunks, sizeof(int) * (E + S), stream, false, a);
+    const size_t smem_count = sizeof(int) * (E + S) + sizeof(unsigned) * 2 * kThreads;
+    err = launch(layout_count_kernel<IdxT>, a.num_chunks, smem_count, stream, false, a);
     if (err != cudaSuccess) return err;
     return launch(assign, a.num_chunks, smem, stream, true, a);
 }

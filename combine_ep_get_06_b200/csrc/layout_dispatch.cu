@@ -122,18 +122,18 @@ __global__ void __launch_bounds__(kThreads) layout_dispatch_kernel(LayoutArgs a,
         reinterpret_cast<uint4*>(zeros)[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
 
-    const SlotRank r = small_layout<IdxT>(a, m, e, bad);
-    const int row_s = slot_row(m, r, E);
-    srow[tid] = (row_s < a.h.max_recv_rows) ? row_s : -1;
-    if (has_slot && (int)(s / k) % G == c_cta) write_slot(a, s, row_s, e, wv);
-    if (c_cta == 0) {
-        write_totals(a, m, E);
-        for (int g = tid; g < S; g += blockDim.x) a.h.seg_tokens[g] = m.seg[g];
+    const int row_s = small_layout<IdxT>(a, m, e, bad, wv);
+    srow[tid] = row_s;
+    {   // this CTA's share of the slot map, the per-row arrays and the padding rows
+        const int64_t n = (int64_t)T * k;
+        if (has_slot && s >= n * c_cta / G && s < n * (c_cta + 1) / G) a.h.slot_map[s] = row_s;
+        const int V = m.lcoff[E];
+        write_rows(a, m, (int)((int64_t)V * c_cta / G), (int)((int64_t)V * (c_cta + 1) / G));
     }
+    if (c_cta == 0) write_totals(a, m, E, S);
     const int P = m.padoff[E];
     const int p0 = (int)((int64_t)P * c_cta / G), p1 = (int)((int64_t)P * (c_cta + 1) / G);
     write_padding(a, m, E, p0, p1);
-    pdl_launch_dependents();
     __syncthreads();
 
     // Padding rows of this CTA's share: bulk copies of zeros.
@@ -186,6 +186,7 @@ __global__ void __launch_bounds__(kThreads) layout_dispatch_kernel(LayoutArgs a,
             }
         }
     }
+    pdl_launch_dependents();
     if (warp == 0) bulk_wait_all();
 }
 
