@@ -98,6 +98,16 @@ ep_status check_handle(const ep_handle* h) {
 
 namespace ep {
 
+ep_status fail(ep_status status, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return status;
+}
+
 int device_sm_count() {
     static std::atomic<int> cache[128];
     int dev = 0;

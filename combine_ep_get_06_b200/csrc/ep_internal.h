@@ -79,4 +79,7 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
 
+// Records a printf-style message for ep_last_error() and returns status.
+ep_status fail(ep_status status, const char* fmt, ...);
+
 }  // namespace ep

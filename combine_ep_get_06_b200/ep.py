@@ -56,6 +56,7 @@ SIGNATURES = {
     "ep_handle_init": (ctypes.c_int, [_HP, _I32, _I32, _I32, _I32, _I32, _I32, _P, _SZ]),
     "ep_layout_workspace_bytes": (_SZ, [_HP]),
     "ep_get_layout": (ctypes.c_int, [_HP, _P, _I32, _P, _P, _P, _P, _SZ, _P]),
+    "ep_get_layout_static": (ctypes.c_int, [_HP, _P, _I32, _P, _P, _P, _P]),
     "ep_dispatch": (ctypes.c_int, [_HP, ctypes.c_int, _P, _P, _I32, _P, _P, _P]),
     "ep_layout_dispatch": (ctypes.c_int, [_HP, _P, _I32, _P, _P, _P, _P, _SZ, ctypes.c_int, _P, _P, _I32,
                                           _P, _P, _P]),

@@ -152,6 +152,28 @@ EP_API ep_status ep_get_layout(ep_handle* handle, const void* topk_idx, int32_t 
                                float* recv_topk_weights, void* workspace,
                                size_t workspace_bytes, ep_stream_t stream);
 
+/* Scratch held by the library for ep_get_layout_static (per GPU). */
+#define EP_STATIC_LAYOUT_SCRATCH_BYTES ((size_t)1 << 20)
+
+/* ep_get_layout without a workspace argument.  The paper has no
+ * counterpart: this entry exists for callers that cannot allocate device
+ * memory themselves -- code running inside a host program that owns every
+ * device allocation (a serving engine with a fixed memory plan), or plain C
+ * code without a device allocator -- and so cannot hand ep_get_layout a
+ * workspace.  The per-chunk histograms go to a fixed array inside this
+ * library instead: EP_STATIC_LAYOUT_SCRATCH_BYTES on every GPU that loads
+ * it, kept until the process exits.  Same arguments (minus the workspace),
+ * results and errors as ep_get_layout, plus EP_ERR_INVALID_ARG when
+ * ep_layout_workspace_bytes(handle) exceeds EP_STATIC_LAYOUT_SCRATCH_BYTES
+ * (for E = 256 experts about a million slots fit).  Allocates and frees
+ * nothing.  The first call on each device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current, so make that
+ * first call before any stream capture.  All calls share the array: calls
+ * that overlap on the GPU race on it. */
+EP_API ep_status ep_get_layout_static(ep_handle* handle, const void* topk_idx, int32_t idx_is_int64,
+                                      const float* topk_weights, int32_t* recv_topk_idx,
+                                      float* recv_topk_weights, ep_stream_t stream);
+
 /* Dispatch (dispatch_forward; with a bf16 gradient and the forward's
  * handle it is combine_backward): row t of x goes to rows slot_map[t*k+j]
  * of recv_x for every valid j, padding rows are zeroed, rows >= R are not
