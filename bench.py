@@ -28,6 +28,7 @@ this path; single-threaded C) on a bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -58,6 +59,8 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default=WORKLOAD, choices=sorted(W.WORKLOADS))
+    p.add_argument("--tokens", type=int, default=None,
+                   help="override the workload's token count (same shapes otherwise; for profiling)")
     p.add_argument("--decode-pairs", type=int, default=256)
     p.add_argument("--decode-replays", type=int, default=20)
     p.add_argument("--e2e-steps", type=int, default=5)
@@ -90,6 +93,24 @@ def step_bytes(w: W.Workload, T: int, V: int, P: int, R: int) -> dict:
         dispatch = T * H * 2 + T * k * 4 + (V + P) * H * 2
     combine = V * H * 2 + T * k * 8 + T * H * 2
     return {"layout": layout, "dispatch": dispatch, "combine": combine}
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest x over all ranks (the slowest rank's time); x itself at N=1."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_gbs(bytes_per_rank_step: int, world: int, ms_per_step: float) -> float:
+    """Whole-job GB/s: every rank moves its own batch's bytes each step, and a
+    step lasts as long as the slowest rank."""
+    return bytes_per_rank_step * world / (ms_per_step * 1e-3) / 1e9
 
 
 # ---------------------------------------------------------------- clocks
@@ -178,6 +199,8 @@ def run_ours(args, rank, world, dev):
     import combine_ep_get_06_b200 as ep
 
     w = W.WORKLOADS[args.workload]
+    if args.tokens is not None:
+        w = dataclasses.replace(w, T=args.tokens)
     inp = W.make_inputs(w, seed=rank)
     y_np = W.make_y(w, seed=rank)
     T, k, H = w.T, w.k, w.H
@@ -249,13 +272,10 @@ def run_ours(args, rank, world, dev):
     com_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
     handle.check_error()
 
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step = total_ms / K
     step_total = sum(nbytes.values())
-    value = step_total * world / (ms_per_step * 1e-3) / 1e9
+    value = weak_scaling_gbs(step_total, world, ms_per_step)
     peak, peak_kind = hbm_peak()
 
     res = {

@@ -6,47 +6,40 @@
 // copies that buffer to each of the token's k receive rows with bulk
 // shared->global copies (cp.async.bulk, never multicast), so the SMs issue
 // a handful of copy instructions per row instead of k stores per 16 bytes.
-// Two row buffers alternate, so quantising row i+1 overlaps the copies of
-// row i.  Padding rows are written by bulk copies of a zeroed buffer, one
-// row per lane of warp 0.  Launched with programmatic dependent launch: a
-// CTA waits for the previous grid before reading anything, and lets the
-// next grid start launching once it has issued all its copies.
+// Two row buffers alternate, so filling row i+1 overlaps the copies of row
+// i, and the loads of a CTA's next row are issued as soon as the current
+// row is in shared memory, so they are in flight across the barrier and
+// the copy issue.  Padding rows are written by bulk copies of a zeroed
+// buffer, one row per lane of warp 0.
 //
 // A CTA walks rows grid-stride: token rows [0, T), then padding batches of
-// 32 rows.  In the quantising mode a 1x128 block is 8 consecutive lanes
-// (16 bf16 values each): its amax is a 3-step xor shuffle, and lane 0 of
-// the group stores the block's scale.
-#include "ep_device.cuh"
-#include "ep_internal.h"
+// 32 rows.  Launched with programmatic dependent launch: a CTA waits for
+// the previous grid before reading anything, and lets the next grid start
+// launching once it has issued all its copies.
+#include "dispatch_device.cuh"
 
 namespace ep {
 namespace {
 
+using namespace dispatch_dev;
+
 constexpr int kThreads = 256;
-constexpr float kE4m3Max = 448.0f;
-constexpr float kAmaxFloor = 1e-4f;
-
-struct Geometry {
-    int row_bytes;     // bytes of one receive row
-    int ipr;           // 16-byte items per receive row
-    int scale_bytes;   // bytes of one row of scales (0 in bf16 mode)
-    int scale_pad;     // scale_bytes rounded up to 16
-};
-
-__host__ __device__ inline Geometry geometry(int mode, int H) {
-    Geometry g;
-    const bool fp8 = mode != EP_X_BF16;
-    g.row_bytes = fp8 ? H : 2 * H;
-    g.ipr = g.row_bytes / 16;
-    g.scale_bytes = fp8 ? (H / 128) * 4 : 0;
-    g.scale_pad = (g.scale_bytes + 15) & ~15;
-    return g;
-}
+constexpr int kPre = 2;  // 32-item slices per warp whose loads are prefetched
 
 // smem: [2][row_bytes] row buffers | [2][scale_pad] scale buffers |
 //       [row_bytes] zeros | [scale_pad] zeros | [2][kMaxTopk] int rows
 __host__ __device__ inline size_t smem_bytes(const Geometry& g) {
     return (size_t)3 * g.row_bytes + (size_t)3 * g.scale_pad + 2 * kMaxTopk * sizeof(int);
+}
+
+template <int kMode>
+__device__ __forceinline__ void prefetch(const DispatchArgs& a, int t, int ipr, Item (&p)[kPre]) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int i = 0; i < kPre; ++i) {
+        const int c = warp * 32 + i * kThreads + lane;
+        p[i] = load_item<kMode>(a, t, c, t < a.T && c < ipr);
+    }
 }
 
 template <int kMode>
@@ -60,7 +53,7 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchArgs a) {
     int* rows_s = (int*)(zeros + geo.row_bytes + geo.scale_pad);   // [2][kMaxTopk]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int T = a.T, k = a.k, H = a.H, B = H / 128;
+    const int T = a.T, k = a.k, B = a.H / 128;
     char* const recv = (char*)a.recv_x;
     char* const rscl = (char*)a.recv_scales;
 
@@ -72,6 +65,8 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchArgs a) {
     pdl_wait();
     const int n_pad = ld_cg(a.num_pad_rows);
     const int n_pad_batches = (n_pad + 31) / 32;
+    Item next[kPre];
+    prefetch<kMode>(a, blockIdx.x, geo.ipr, next);
     __syncthreads();
 
     int it = 0;  // token rows handled by this CTA (selects the buffer)
@@ -86,9 +81,9 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchArgs a) {
                     if (a.bulk_scales)
                         bulk_s2g(rscl + (size_t)row * geo.scale_bytes, zeros + geo.row_bytes, geo.scale_bytes);
                     bulk_commit();
+                    if (kFp8Out && !a.bulk_scales)
+                        for (int b = 0; b < B; ++b) a.recv_scales[(size_t)row * B + b] = 0.0f;
                 }
-                if (kFp8Out && !a.bulk_scales && row >= 0 && row < a.max_rows)
-                    for (int b = 0; b < B; ++b) a.recv_scales[(size_t)row * B + b] = 0.0f;
             }
             continue;
         }
@@ -106,44 +101,18 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchArgs a) {
 
         if (tid < k) rows[tid] = ld_cg(a.slot_map + (size_t)t * k + tid);
 
-        // Fill the row buffer: warp-uniform loop over 32-item slices.
-        for (int c0 = warp * 32; c0 < geo.ipr; c0 += kThreads) {
-            const int c = c0 + lane;
-            const bool active = c < geo.ipr;
-            if (kMode == EP_X_BF16_TO_FP8) {
-                const char* src = (const char*)a.x + (size_t)t * H * 2 + (size_t)c * 32;
-                uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
-                if (active) {
-                    v0 = ld_stream(src);
-                    v1 = ld_stream(src + 16);
-                }
-                float f[16] = {bf16_lo(v0.x), bf16_hi(v0.x), bf16_lo(v0.y), bf16_hi(v0.y),
-                               bf16_lo(v0.z), bf16_hi(v0.z), bf16_lo(v0.w), bf16_hi(v0.w),
-                               bf16_lo(v1.x), bf16_hi(v1.x), bf16_lo(v1.y), bf16_hi(v1.y),
-                               bf16_lo(v1.z), bf16_hi(v1.z), bf16_lo(v1.w), bf16_hi(v1.w)};
-                float amax = 0.0f;
+        // Fill the row buffer: the prefetched slices, then any further ones.
 #pragma unroll
-                for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
-                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-                amax = fmaxf(amax, kAmaxFloor);
-                const float scale = __fdiv_rn(amax, kE4m3Max);
-                const float inv = __fdiv_rn(kE4m3Max, amax);
-                uint32_t w[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    w[i] = pack_e4m3x2(__fmul_rn(f[4 * i], inv), __fmul_rn(f[4 * i + 1], inv)) |
-                           (pack_e4m3x2(__fmul_rn(f[4 * i + 2], inv), __fmul_rn(f[4 * i + 3], inv)) << 16);
-                if (active) {
-                    reinterpret_cast<uint4*>(rb)[c] = make_uint4(w[0], w[1], w[2], w[3]);
-                    if ((c & 7) == 0) sb[c >> 3] = scale;
-                }
-            } else if (active) {
-                reinterpret_cast<uint4*>(rb)[c] = ld_stream((const char*)a.x + (size_t)t * geo.row_bytes + (size_t)c * 16);
-                if (kMode == EP_X_FP8 && (c & 7) == 0) sb[c >> 3] = ld_cg(a.x_scales + (size_t)t * B + (c >> 3));
-            }
+        for (int i = 0; i < kPre; ++i) {
+            const int c0 = warp * 32 + i * kThreads;
+            if (c0 < geo.ipr) fill_item<kMode>(a, t, c0 + lane, c0 + lane < geo.ipr, next[i], rb, sb);
         }
+        for (int c0 = warp * 32 + kPre * kThreads; c0 < geo.ipr; c0 += kThreads) {
+            const int c = c0 + lane;
+            fill_item<kMode>(a, t, c, c < geo.ipr, load_item<kMode>(a, t, c, c < geo.ipr), rb, sb);
+        }
+        // This CTA's next token row: its loads fly across the barrier and copy issue.
+        prefetch<kMode>(a, r + gridDim.x, geo.ipr, next);
         fence_proxy_async_smem();
         __syncthreads();
 

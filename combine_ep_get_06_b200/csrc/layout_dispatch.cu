@@ -8,17 +8,18 @@
 // writes their slot-map entries and per-row arrays, quantises or copies
 // their x rows into a shared row buffer and bulk-copies (TMA, no multicast)
 // that buffer to the k receive rows; it also writes its share of the
-// padding rows.  Each CTA loads the x row of its first token before the
-// layout, so that load overlaps the layout's latency.
+// padding rows.  Each CTA loads and quantises the x row of its first token
+// before the layout, so that work overlaps the layout's latency.
+#include "dispatch_device.cuh"
 #include "layout_device.cuh"
 
 namespace ep {
 namespace {
 
 using namespace layout_dev;
-
-constexpr float kE4m3Max = 448.0f;
-constexpr float kAmaxFloor = 1e-4f;
+using dispatch_dev::Item;
+using dispatch_dev::fill_item;
+using dispatch_dev::load_item;
 
 struct FusedGeometry {
     int row_bytes, ipr, scale_bytes, scale_pad;
@@ -39,53 +40,6 @@ __host__ __device__ inline FusedGeometry fused_geometry(int mode, int H, int E, 
     g.srow_off = g.zero_off + g.row_bytes + g.scale_pad;
     g.total = g.srow_off + sizeof(int) * kThreads;
     return g;
-}
-
-// Quantises (or copies) item c of token t's row into the row buffer.
-template <int kMode>
-__device__ __forceinline__ void fill_item(const DispatchArgs& d, int t, int c, bool active, uint4 v0, uint4 v1,
-                                          unsigned char* rb, float* sb) {
-    if (kMode == EP_X_BF16_TO_FP8) {
-        float f[16] = {bf16_lo(v0.x), bf16_hi(v0.x), bf16_lo(v0.y), bf16_hi(v0.y),
-                       bf16_lo(v0.z), bf16_hi(v0.z), bf16_lo(v0.w), bf16_hi(v0.w),
-                       bf16_lo(v1.x), bf16_hi(v1.x), bf16_lo(v1.y), bf16_hi(v1.y),
-                       bf16_lo(v1.z), bf16_hi(v1.z), bf16_lo(v1.w), bf16_hi(v1.w)};
-        float amax = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-        amax = fmaxf(amax, kAmaxFloor);
-        const float scale = __fdiv_rn(amax, kE4m3Max);
-        const float inv = __fdiv_rn(kE4m3Max, amax);
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            w[i] = pack_e4m3x2(__fmul_rn(f[4 * i], inv), __fmul_rn(f[4 * i + 1], inv)) |
-                   (pack_e4m3x2(__fmul_rn(f[4 * i + 2], inv), __fmul_rn(f[4 * i + 3], inv)) << 16);
-        if (active) {
-            reinterpret_cast<uint4*>(rb)[c] = make_uint4(w[0], w[1], w[2], w[3]);
-            if ((c & 7) == 0) sb[c >> 3] = scale;
-        }
-    } else if (active) {
-        reinterpret_cast<uint4*>(rb)[c] = v0;
-        if (kMode == EP_X_FP8 && (c & 7) == 0) sb[c >> 3] = __ldg(d.x_scales + (size_t)t * (d.H / 128) + (c >> 3));
-    }
-}
-
-template <int kMode>
-__device__ __forceinline__ void load_item(const DispatchArgs& d, int t, int c, bool active, uint4& v0, uint4& v1) {
-    v0 = v1 = make_uint4(0, 0, 0, 0);
-    if (!active) return;
-    if (kMode == EP_X_BF16_TO_FP8) {
-        const char* src = (const char*)d.x + (size_t)t * d.H * 2 + (size_t)c * 32;
-        v0 = ld_stream(src);
-        v1 = ld_stream(src + 16);
-    } else {
-        const size_t rb = kMode == EP_X_BF16 ? (size_t)d.H * 2 : (size_t)d.H;
-        v0 = ld_stream((const char*)d.x + (size_t)t * rb + (size_t)c * 16);
-    }
 }
 
 template <typename IdxT, int kMode>
@@ -115,11 +69,19 @@ __global__ void __launch_bounds__(kThreads) layout_dispatch_kernel(LayoutArgs a,
         e = read_expert((const IdxT*)a.topk_idx, s, E, bad);
         if (a.topk_weights) wv = __ldg(a.topk_weights + s);
     }
-    uint4 pre0, pre1;
-    const bool first_active = c_cta < T && tid < geo.ipr;
-    load_item<kMode>(d, c_cta, tid, first_active, pre0, pre1);
+    const Item pre = load_item<kMode>(d, c_cta, tid, c_cta < T && tid < geo.ipr);
     for (int i = tid; i < (geo.row_bytes + geo.scale_pad) / 16; i += kThreads)
         reinterpret_cast<uint4*>(zeros)[i] = make_uint4(0, 0, 0, 0);
+    // The first token row needs no routing: quantise (or copy) it into the
+    // row buffer now, so that work overlaps the layout below.
+    if (c_cta < T) {
+        for (int c0 = warp * 32; c0 < geo.ipr; c0 += kThreads) {
+            const int c = c0 + lane;
+            const bool active = c < geo.ipr;
+            const Item it = c0 == warp * 32 ? pre : load_item<kMode>(d, c_cta, c, active);
+            fill_item<kMode>(d, c_cta, c, active, it, rb, sb);
+        }
+    }
     fence_proxy_async_smem();
 
     const int row_s = small_layout<IdxT>(a, m, e, bad, wv);
@@ -149,27 +111,18 @@ __global__ void __launch_bounds__(kThreads) layout_dispatch_kernel(LayoutArgs a,
         }
     }
 
-    bool first = true;
     for (int t = c_cta; t < T; t += G) {
-        if (!first) {
+        if (t != c_cta) {   // the first row is already in the buffer
             if (warp == 0) bulk_wait_read<0>();
             __syncthreads();
-        }
-        for (int c0 = warp * 32; c0 < geo.ipr; c0 += kThreads) {
-            const int c = c0 + lane;
-            const bool active = c < geo.ipr;
-            uint4 v0, v1;
-            if (first && c0 == warp * 32) {
-                v0 = pre0;
-                v1 = pre1;
-            } else {
-                load_item<kMode>(d, t, c, active, v0, v1);
+            for (int c0 = warp * 32; c0 < geo.ipr; c0 += kThreads) {
+                const int c = c0 + lane;
+                const bool active = c < geo.ipr;
+                fill_item<kMode>(d, t, c, active, load_item<kMode>(d, t, c, active), rb, sb);
             }
-            fill_item<kMode>(d, t, c, active, v0, v1, rb, sb);
+            fence_proxy_async_smem();
+            __syncthreads();
         }
-        first = false;
-        fence_proxy_async_smem();
-        __syncthreads();
         if (warp == 0 && lane < k) {
             const int row = srow[t * k + lane];
             if (row >= 0) {
