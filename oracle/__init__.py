@@ -24,9 +24,11 @@ X_BF16, X_FP8_PREQUANT, X_BF16_QUANT_FP8 = 0, 1, 2
 
 
 def lib():
+    """The oracle library.  EP_ORACLE_LIB names another build of it (the
+    mutation tests load deliberately broken copies that way)."""
     global _lib
     if _lib is None:
-        path = _build.build()
+        path = os.environ.get("EP_ORACLE_LIB") or _build.build()
         L = ctypes.CDLL(path)
         P = ctypes.c_void_p
         i32, i64, u32 = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32
@@ -133,18 +135,22 @@ def layout(topk_idx: np.ndarray, E: int, S: int, align: int, topk_weights=None,
 
 # ----------------------------------------------------------------- dispatch
 
+UNWRITTEN = 0x5A  # every byte of the dispatch outputs starts as this
+
+
 def dispatch(lay: dict, x: np.ndarray, mode: int, x_scales=None):
     """Returns (recv_x [max_rows, H], recv_scales [max_rows, H/128] or None).
-    Rows >= R are left zero-initialised (the oracle never writes them)."""
+    Every output byte starts as UNWRITTEN, so rows the oracle does not
+    write (rows >= R) keep it and a missing write shows."""
     T, k, cap, R = lay["T"], lay["k"], lay["max_rows"], lay["R"]
     if mode == X_BF16:
         x = _c(x, np.uint16)
-        recv = np.zeros((cap, x.shape[1]), np.uint16)
+        recv = np.full((cap, x.shape[1]), UNWRITTEN * 0x0101, np.uint16)
         scales = None
     else:
         x = _c(x, np.uint8 if mode == X_FP8_PREQUANT else np.uint16)
-        recv = np.zeros((cap, x.shape[1]), np.uint8)
-        scales = np.zeros((cap, x.shape[1] // 128), np.float32)
+        recv = np.full((cap, x.shape[1]), UNWRITTEN, np.uint8)
+        scales = np.full((cap, x.shape[1] // 128), UNWRITTEN * 0x01010101, np.uint32).view(np.float32)
     H = x.shape[1]
     xs = None if x_scales is None else _c(x_scales, np.float32)
     lib().oracle_dispatch(mode, T, k, H, R, _p(lay["slot_map"]), _p(lay["recv_src"]), _p(x),

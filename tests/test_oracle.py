@@ -360,6 +360,40 @@ def test_combine_equals_exact_rational_fma_chain():
         assert np.array_equal(out, bf16_bits_of(exp))
 
 
+def test_combine_near_cancellation_equals_exact_rational_fma_chain():
+    # Sums that nearly cancel: the result is tiny next to its terms, so every
+    # binary32 rounding step, and the order of the steps, reaches the bf16
+    # output.  Each token's last weight is chosen to cancel the others.
+    rng = np.random.default_rng(17)
+    T, k, H, E = 64, 4, 8, 16
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int64)
+    lay = oracle.layout(idx, E, 1, 1)
+    y = bf16_bits_of(rng.uniform(0.5, 2.0, (lay["max_rows"], H)) * rng.choice([-1, 1], (lay["max_rows"], H)))
+    yf = f32_of_bf16(y).astype(np.float64)
+    sm = lay["slot_map"].reshape(T, k)
+    w = rng.uniform(-2, 2, (T, k)).astype(np.float32)
+    for t in range(T):           # w[t,k-1] * y[last, 0] ~ -(sum of the others at column 0)
+        part = sum(float(w[t, j]) * yf[sm[t, j], 0] for j in range(k - 1))
+        w[t, k - 1] = np.float32(-part / yf[sm[t, k - 1], 0] * (1 + rng.uniform(-1e-5, 1e-5)))
+    out, _ = oracle.combine(lay["slot_map"], T, k, y, w)
+    exp = np.empty((T, H), np.float32)
+    for t in range(T):
+        for h in range(H):
+            acc = Fraction(0)
+            for j in range(k):
+                acc = round_fraction(Fraction(float(w[t, j])) * Fraction(float(yf[sm[t, j], h])) + acc, 24)
+            exp[t, h] = float(round_fraction(acc, 8))
+    assert np.array_equal(out, bf16_bits_of(exp))
+    # the case is sensitive: two roundings per step, or the reverse order, changes the bf16 result
+    twice = np.empty(T, np.float32)
+    for t in range(T):
+        acc = Fraction(0)
+        for j in range(k):
+            acc = round_fraction(round_fraction(Fraction(float(w[t, j])) * Fraction(float(yf[sm[t, j], 0])), 24) + acc, 24)
+        twice[t] = float(round_fraction(acc, 8))
+    assert not np.array_equal(bf16_bits_of(twice), out[:, 0])
+
+
 def test_combine_of_identity_outputs_returns_x():
     w = W.WORKLOADS["mid"]
     inp = W.make_inputs(w, seed=3, T=256)
