@@ -13,6 +13,8 @@
 //              chunk while count still runs, then waits, reduces the
 //              histograms of all chunks, scans the aligned expert sizes and
 //              writes its slots and its share of the padding rows.
+// Every layout kernel is launched with programmatic dependent launch and
+// touches global memory only after waiting for the grid before it.
 #include "layout_device.cuh"
 
 namespace ep {
@@ -27,6 +29,10 @@ __global__ void __launch_bounds__(kThreads) layout_single_kernel(LayoutArgs a) {
     Smem m(smem_raw, E, S);
     const int64_t s = threadIdx.x;
     const bool has_slot = s < (int64_t)a.h.num_tokens * a.h.num_topk;
+    // Launched with programmatic dependent launch: nothing global is read
+    // or written before the previous grid (which may produce topk_idx or
+    // still read the handle) has finished.
+    pdl_wait();
     bool bad = false;
     int e = -1;
     float wv = 0.0f;
@@ -55,17 +61,21 @@ __global__ void __launch_bounds__(kThreads) layout_count_kernel(LayoutArgs a) {
     const int64_t s = (int64_t)t0 * k + tid;
     const IdxT* idx = (const IdxT*)a.topk_idx;
 
+    // Programmatic dependent launch: wait for the previous grid before any
+    // global access; only then let the assign pass start (it reads topk_idx
+    // before waiting on this grid).
+    pdl_wait();
+    pdl_launch_dependents();
     bool bad = false;
     int e = -1;
     if (s < (int64_t)t1 * k) e = read_expert(idx, s, E, bad);
-    pdl_launch_dependents();
     for (int i = tid; i < E + S; i += blockDim.x) smem_raw[i] = 0;
     tmask[2 * tid] = 0;
     tmask[2 * tid + 1] = 0;
     if (bad) atomicOr(a.h.error_word, EP_DEVERR_BAD_TOPK_IDX);
     __syncthreads();
     if (e >= 0) atomicAdd(&hist[e], 1);
-    if (S <= 64) mark_segment(tmask, tid / k, e, E, S);
+    if (S <= 64) mark_segment(tmask, tid / k, e, E, S, k);
     else count_segments_walk(idx, t0, t1, k, E, S, seg);
     __syncthreads();
     if (S <= 64) {
@@ -157,9 +167,9 @@ cudaError_t launch_layout_t(const LayoutArgs& a, cudaStream_t stream) {
         if ((err = cudaFuncSetAttribute(assign, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
             return err;
     }
-    if (a.num_chunks == 1) return launch(single, 1, smem, stream, false, a);
+    if (a.num_chunks == 1) return launch(single, 1, smem, stream, true, a);
     const size_t smem_count = sizeof(int) * (E + S) + sizeof(unsigned) * 2 * kThreads;
-    err = launch(layout_count_kernel<IdxT>, a.num_chunks, smem_count, stream, false, a);
+    err = launch(layout_count_kernel<IdxT>, a.num_chunks, smem_count, stream, true, a);
     if (err != cudaSuccess) return err;
     return launch(assign, a.num_chunks, smem, stream, true, a);
 }

@@ -60,18 +60,36 @@ __device__ __forceinline__ void count_segments_walk(const IdxT* idx, int t0, int
     }
 }
 
-// S <= 64: the slot's thread sets bit g of its token's mask (two 32-bit
-// words per token).
-__device__ __forceinline__ void mark_segment(unsigned* tmask, int token, int e, int E, int S) {
-    if (e < 0) return;
-    const int g = e / (E / S);
-    atomicOr(&tmask[2 * token + (g >> 5)], 1u << (g & 31));
+// S <= 64: records in tmask (two 32-bit words per token) the segments the
+// token's slots reach.  When k divides 32 a token's k slots are k
+// consecutive lanes: their bits are OR-reduced with shuffles and the first
+// lane stores them (no atomics); otherwise each slot ORs in its own bit.
+// All lanes of the warp must call it.
+__device__ __forceinline__ void mark_segment(unsigned* tmask, int token, int e, int E, int S, int k) {
+    const int g = e >= 0 ? e / (E / S) : 0;
+    unsigned lo = (e >= 0 && g < 32) ? 1u << g : 0u;
+    unsigned hi = (e >= 0 && g >= 32) ? 1u << (g - 32) : 0u;
+    if ((32 % k) == 0) {
+        for (int o = 1; o < k; o <<= 1) {
+            lo |= __shfl_xor_sync(0xffffffffu, lo, o);
+            hi |= __shfl_xor_sync(0xffffffffu, hi, o);
+        }
+        if ((threadIdx.x & 31) % k == 0) {
+            tmask[2 * token] = lo;
+            tmask[2 * token + 1] = hi;
+        }
+    } else if (e >= 0) {
+        atomicOr(&tmask[2 * token + (g >> 5)], g < 32 ? lo : hi);
+    }
 }
 
-// S <= 64: tokens per segment from the masks of n_tokens tokens, one
-// ballot per segment and warp, one atomic per (warp, segment).
+// S <= 64: tokens per segment from the masks of n_tokens tokens.  Per warp
+// of 32 tokens, one ballot per segment; lane g keeps segment g's count in a
+// register and all lanes then add theirs at once (one atomic per lane, so
+// no lane waits on a chain of atomics).
 __device__ __forceinline__ void count_segments_masks(const unsigned* tmask, int n_tokens, int S, int* seg) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int mine_lo = 0, mine_hi = 0;  // counts of segments lane and 32 + lane
     for (int t0 = warp * 32; t0 < n_tokens; t0 += kThreads) {
         const int t = t0 + lane;
         const unsigned lo = t < n_tokens ? tmask[2 * t] : 0u;
@@ -79,9 +97,12 @@ __device__ __forceinline__ void count_segments_masks(const unsigned* tmask, int 
         for (int g = 0; g < S; ++g) {
             const unsigned bit = g < 32 ? (lo >> g) & 1u : (hi >> (g - 32)) & 1u;
             const int n = __popc(__ballot_sync(0xffffffffu, bit));
-            if (lane == 0 && n) atomicAdd(&seg[g], n);
+            if (g < 32) mine_lo += lane == g ? n : 0;
+            else mine_hi += lane == g - 32 ? n : 0;
         }
     }
+    if (lane < S && mine_lo) atomicAdd(&seg[lane], mine_lo);
+    if (32 + lane < S && mine_hi) atomicAdd(&seg[32 + lane], mine_hi);
 }
 
 // -------------------------------------------------------------- block scans
@@ -352,7 +373,7 @@ __device__ __forceinline__ int small_layout(const LayoutArgs& a, Smem& m, int e,
     if (bad) atomicOr(a.h.error_word, EP_DEVERR_BAD_TOPK_IDX);
     __syncthreads();
     mark_slot(e, m.tab, E);
-    if (S <= 64) mark_segment(m.tmask, tid / k, e, E, S);
+    if (S <= 64) mark_segment(m.tmask, tid / k, e, E, S, k);
     __syncthreads();
     const int wrank = rank_in_warp(e, m.tab, E);
     if (S <= 64) count_segments_masks(m.tmask, T, S, m.seg);

@@ -61,7 +61,10 @@ __global__ void __launch_bounds__(kThreads) layout_dispatch_kernel(LayoutArgs a,
     char* const recv = (char*)d.recv_x;
     char* const rscl = (char*)d.recv_scales;
 
-    // Loads first: this thread's slot, and its item of the first token row.
+    // Launched with programmatic dependent launch: wait for the previous
+    // grid before touching global memory.  Then the loads: this thread's
+    // slot, and its item of the first token row.
+    pdl_wait();
     bool bad = false;
     int e = -1;
     float wv = 0.0f;
@@ -156,6 +159,11 @@ cudaError_t launch_t(const LayoutArgs& a, const DispatchArgs& d, cudaStream_t st
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = g.total;
     cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kernel, a, d);
 }
 
