@@ -54,6 +54,8 @@ def lib():
         L.oracle_dispatch.restype = None
         L.oracle_combine.argtypes = [i32, i32, i32, P, P, P, P, P, P]
         L.oracle_combine.restype = None
+        L.oracle_combine_backward.argtypes = [i32, i32, i32, i32, P, P, P, P, P, P, P]
+        L.oracle_combine_backward.restype = None
         _lib = L
     return _lib
 
@@ -172,3 +174,18 @@ def combine(slot_map: np.ndarray, T: int, k: int, y: np.ndarray, weights=None,
     ow = np.empty((T, k), np.float32) if want_out_weights else None
     lib().oracle_combine(T, k, H, _p(sm), _p(y), _p(w), _p(rw), _p(ow), _p(out))
     return out, ow
+
+
+def combine_backward(lay: dict, grad_out: np.ndarray, y: np.ndarray, weights: np.ndarray):
+    """Backward of the weighted combine.  Returns (grad_y bf16 bits
+    [max_rows, H] -- rows >= R keep UNWRITTEN --, grad_w float64 [T, k])."""
+    T, k, cap, R = lay["T"], lay["k"], lay["max_rows"], lay["R"]
+    g = _c(grad_out, np.uint16)
+    yy = _c(y, np.uint16)
+    w = _c(weights, np.float32)
+    H = g.shape[1]
+    grad_y = np.full((cap, H), UNWRITTEN * 0x0101, np.uint16)
+    grad_w = np.empty((T, k), np.float64)
+    lib().oracle_combine_backward(T, k, H, R, _p(lay["slot_map"]), _p(lay["recv_src"]), _p(g), _p(yy),
+                                  _p(w), _p(grad_y), _p(grad_w))
+    return grad_y, grad_w

@@ -25,7 +25,12 @@
  *   - combine: the k expert outputs of each token gathered back and summed
  *     (combine_forward), weighted by topk_weights; with no weights it is
  *     the adjoint of dispatch (dispatch_backward), optionally gathering the
- *     per-row weight gradient back to [T, k].
+ *     per-row weight gradient back to [T, k];
+ *   - the backward of the weighted combine (combine_backward, which the
+ *     page runs as a dispatch of the output gradient): each receive row gets
+ *     its slot's weight times the token's output gradient, and each slot's
+ *     weight gradient is the dot product of the token's output gradient with
+ *     the row's expert output.
  *
  * Readings taken where the pages are silent (each is a definition here):
  *   - rows of one expert are ordered by flat slot s = t*k + j, ascending;
@@ -41,7 +46,12 @@
  *     scale = amax / 448, inv = 448 / amax (two IEEE divisions),
  *     q = e4m3(x * inv) rounded to nearest-even with saturation to +-448;
  *   - combine: acc = +0.0f, then for j = 0..k-1 over valid slots
- *     acc = fmaf(w[t,j], y[row], acc), and one bf16 rounding at the end.
+ *     acc = fmaf(w[t,j], y[row], acc), and one bf16 rounding at the end;
+ *   - combine backward: grad_y[row] = bf16(w * g) with the product taken in
+ *     binary32 (one multiply, one bf16 rounding); padding rows of grad_y are
+ *     zero; grad_w is the exact dot product, accumulated here in binary64
+ *     (the GPU accumulates in binary32; tests bound the difference by the
+ *     binary32 summation error bound).
  *
  * Parity pins: every function here is checked against brute force,
  * independent library routines, exact rational arithmetic or invariants
@@ -303,4 +313,33 @@ EXPORT void oracle_combine(int32_t T, int32_t k, int32_t H, const int32_t* slot_
                 out_weights[(int64_t)t * k + j] =
                     (sm[j] >= 0 && recv_weights_in) ? recv_weights_in[sm[j]] : 0.0f;
     }
+}
+
+/* ------------------------------------------------------- combine backward */
+
+/* Backward of the weighted combine, for the output gradient g [T,H] bf16:
+ *   grad_y[slot_map[t*k+j], h] = bf16(w[t,j] * g[t,h])   (binary32 product)
+ *   grad_w[t,j] = sum_h g[t,h] * y[slot_map[t*k+j], h]   (binary64; 0 when dropped)
+ * and grad_y rows r < R with recv_src[r] < 0 (padding) are zero. */
+EXPORT void oracle_combine_backward(int32_t T, int32_t k, int32_t H, int32_t R, const int32_t* slot_map,
+                                    const int32_t* recv_src, const uint16_t* g, const uint16_t* y,
+                                    const float* weights, uint16_t* grad_y, double* grad_w) {
+    for (int32_t t = 0; t < T; ++t)
+        for (int32_t j = 0; j < k; ++j) {
+            int32_t row = slot_map[(int64_t)t * k + j];
+            if (row < 0) {
+                grad_w[(int64_t)t * k + j] = 0.0;
+                continue;
+            }
+            float w = weights[(int64_t)t * k + j];
+            double dot = 0.0;
+            for (int32_t h = 0; h < H; ++h) {
+                float gv = oracle_bf16_to_f32(g[(size_t)t * H + h]);
+                grad_y[(size_t)row * H + h] = oracle_f32_to_bf16(w * gv);
+                dot += (double)gv * (double)oracle_bf16_to_f32(y[(size_t)row * H + h]);
+            }
+            grad_w[(int64_t)t * k + j] = dot;
+        }
+    for (int32_t row = 0; row < R; ++row)
+        if (recv_src[row] < 0) memset(grad_y + (size_t)row * H, 0, sizeof(uint16_t) * H);
 }

@@ -460,6 +460,65 @@ def test_combine_token_with_no_valid_slot_is_positive_zero():
     assert ow.tolist() == [[0, 0, 0], [0, 7.0, 0]]
 
 
+# ------------------------------------------------------ combine backward
+
+def test_combine_backward_matches_library_gather_and_dot():
+    rng = np.random.default_rng(23)
+    T, k, H, E, a = 48, 4, 64, 12, 3
+    idx = rng.integers(0, E, size=(T, k)).astype(np.int64)
+    idx[rng.random((T, k)) < 0.2] = -1
+    w = rng.standard_normal((T, k)).astype(np.float32)
+    lay = oracle.layout(idx, E, 4, a, w)
+    g = bf16_bits_of(rng.standard_normal((T, H)))
+    y = bf16_bits_of(rng.standard_normal((lay["max_rows"], H)))
+    gy, gw = oracle.combine_backward(lay, g, y, w)
+    R, sm = lay["R"], lay["slot_map"].reshape(T, k)
+    gf, yf = f32_of_bf16(g), f32_of_bf16(y)
+    for t in range(T):
+        for j in range(k):
+            r = sm[t, j]
+            if r < 0:
+                assert gw[t, j] == 0.0
+                continue
+            # numpy binary32 multiply, torch's bf16 cast
+            assert np.array_equal(gy[r], bf16_bits_of(np.float32(w[t, j]) * gf[t]))
+            assert np.isclose(gw[t, j], np.dot(gf[t].astype(np.float64), yf[r].astype(np.float64)),
+                              rtol=1e-12, atol=1e-12)
+    pad = lay["recv_src"][:R] < 0
+    assert np.all(gy[:R][pad] == 0)
+    assert np.all(gy[R:] == oracle.UNWRITTEN * 0x0101)
+
+
+def test_combine_backward_is_the_derivative_of_the_weighted_combine():
+    # small integers: every value and sum is exact, so finite differences are exact
+    rng = np.random.default_rng(29)
+    T, k, H, E, a = 20, 3, 16, 7, 2
+    idx = rng.integers(0, E, size=(T, k)).astype(np.int64)
+    idx[rng.random((T, k)) < 0.15] = -1
+    w = rng.integers(-3, 4, size=(T, k)).astype(np.float32)
+    lay = oracle.layout(idx, E, 1, a, w)
+    y = bf16_bits_of(rng.integers(-4, 5, size=(lay["max_rows"], H)))
+    g = bf16_bits_of(rng.integers(-4, 5, size=(T, H)))
+    gf = f32_of_bf16(g).astype(np.int64)
+
+    def loss(weights):      # <combine(y, weights), g>
+        out, _ = oracle.combine(lay["slot_map"], T, k, y, weights)
+        return int((f32_of_bf16(out).astype(np.int64) * gf).sum())
+
+    gy, gw = oracle.combine_backward(lay, g, y, w)
+    base = loss(w)
+    for t in range(T):
+        for j in range(k):
+            w2 = w.copy()
+            w2[t, j] += 1.0
+            assert loss(w2) - base == gw[t, j]          # d loss / d w[t,j]
+    # adjoint in y: <combine(y), g> = <y, grad_y> over the real rows
+    R = lay["R"]
+    real = lay["recv_src"][:R] >= 0
+    lhs = int((f32_of_bf16(y)[:R][real].astype(np.int64) * f32_of_bf16(gy)[:R][real].astype(np.int64)).sum())
+    assert lhs == base
+
+
 # ------------------------------------------------------------- workloads
 
 def test_workloads_are_seeded_and_shaped():

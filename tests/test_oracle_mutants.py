@@ -49,6 +49,12 @@ MUTANTS = {
                              "acc = w * oracle_bf16_to_f32(y[(size_t)sm[j] * H + h]) + acc;"),
     "combine truncates to bf16": ("out[(size_t)t * H + h] = oracle_f32_to_bf16(acc);",
                                   "{ uint32_t u; memcpy(&u, &acc, 4); out[(size_t)t * H + h] = (uint16_t)(u >> 16); }"),
+    "backward drops the weight": ("grad_y[(size_t)row * H + h] = oracle_f32_to_bf16(w * gv);",
+                                  "grad_y[(size_t)row * H + h] = oracle_f32_to_bf16(gv);"),
+    "backward dot uses the token's own row": ("dot += (double)gv * (double)oracle_bf16_to_f32(y[(size_t)row * H + h]);",
+                                              "dot += (double)gv * (double)oracle_bf16_to_f32(y[(size_t)t * H + h]);"),
+    "backward padding not zeroed": ("if (recv_src[row] < 0) memset(grad_y + (size_t)row * H, 0, sizeof(uint16_t) * H);",
+                                    "if (recv_src[row] < 0) {}"),
     "weight gather ignores the slot map": ("(sm[j] >= 0 && recv_weights_in) ? recv_weights_in[sm[j]] : 0.0f;",
                                            "(sm[j] >= 0 && recv_weights_in) ? recv_weights_in[j] : 0.0f;"),
 }
