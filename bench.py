@@ -305,6 +305,27 @@ def run_ours(args, rank, world, dev):
                        "frac": round(achieved / peak, 4), "traffic": combine_traffic(),
                        "algorithmic_bytes": nbytes["combine"]}
 
+    # the backward of the weighted combine (training), same workload
+    gy = torch.empty(rows, H, dtype=torch.bfloat16, device=dev)
+    gw = torch.empty(T, k, dtype=torch.float32, device=dev)
+    g_out = out  # any [T,H] bf16 gradient; the forward's output serves
+    bwd = lambda: ep.combine_backward(g_out, y, handle, wts, grad_y=gy, grad_weights=gw)
+    for _ in range(3):
+        bwd()
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_b = max(3, min(50, K))
+    b0.record(stream)
+    for _ in range(n_b):
+        bwd()
+    b1.record(stream)
+    torch.cuda.synchronize(dev)
+    bwd_ms = b0.elapsed_time(b1) / n_b
+    bwd_bytes = T * H * 2 + V * H * 2 + (V + P) * H * 2 + T * k * 12
+    res["combine_backward"] = {"us": round(bwd_ms * 1e3, 2), "bytes": bwd_bytes,
+                               "gbs": round(bwd_bytes / (bwd_ms * 1e-3) / 1e9, 1),
+                               "frac_of_peak": round(bwd_bytes / (bwd_ms * 1e-3) / 1e9 / peak, 4)}
+    handle.check_error()
+
     if not args.no_decode:
         res["decode"] = run_decode(args, dev)
     if not args.no_e2e:

@@ -337,6 +337,39 @@ EP_API ep_status ep_combine(const ep_handle* h, const void* y, int32_t H, const 
     return ok();
 }
 
+EP_API ep_status ep_combine_backward(const ep_handle* h, const void* grad_out, const void* y, int32_t H,
+                                     const float* topk_weights, void* grad_y, float* grad_weights,
+                                     ep_stream_t stream) {
+    ep_status st = check_handle(h);
+    if (st != EP_OK) return st;
+    if (H < 1 || H % 8 != 0) return invalid("hidden %d must be a positive multiple of 8", H);
+    if (h->num_tokens > 0 && (grad_out == nullptr || !aligned(grad_out, 16)))
+        return invalid("grad_out must be non-NULL and 16-byte aligned");
+    if (y == nullptr || !aligned(y, 16)) return invalid("y must be non-NULL and 16-byte aligned");
+    if (grad_y == nullptr || !aligned(grad_y, 16)) return invalid("grad_y must be non-NULL and 16-byte aligned");
+    if (h->num_tokens > 0 && (grad_weights == nullptr || !aligned(grad_weights, 4)))
+        return invalid("grad_weights must be non-NULL and 4-byte aligned");
+    if (topk_weights && !aligned(topk_weights, 4)) return invalid("topk_weights misaligned");
+    ep::CombineBackwardArgs a;
+    a.grad_out = grad_out;
+    a.y = y;
+    a.topk_weights = topk_weights;
+    a.grad_y = grad_y;
+    a.grad_weights = grad_weights;
+    a.slot_map = h->slot_map;
+    a.pad_rows = h->pad_rows;
+    a.num_pad_rows = h->num_pad_rows;
+    a.error_word = h->error_word;
+    a.T = h->num_tokens;
+    a.k = h->num_topk;
+    a.H = H;
+    a.max_rows = h->max_recv_rows;
+    a.max_pad_rows = h->num_experts * (h->expert_alignment - 1);
+    cudaError_t err = ep::launch_combine_backward(a, (cudaStream_t)stream);
+    if (err != cudaSuccess) return cuda_failed("combine backward launch", err);
+    return ok();
+}
+
 EP_API ep_status ep_read_total_rows(const ep_handle* h, int32_t* total_rows, ep_stream_t stream) {
     ep_status st = check_handle(h);
     if (st != EP_OK) return st;

@@ -76,6 +76,21 @@ struct CombineArgs {
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
 
+struct CombineBackwardArgs {
+    const void* grad_out;            // [T,H] bf16
+    const void* y;                   // [max_rows,H] bf16
+    const float* topk_weights;       // [T,k] or nullable (all 1)
+    void* grad_y;                    // [max_rows,H] bf16
+    float* grad_weights;             // [T,k]
+    const int32_t* slot_map;
+    const int32_t* pad_rows;
+    const int32_t* num_pad_rows;
+    uint32_t* error_word;
+    int32_t T, k, H, max_rows, max_pad_rows;
+};
+
+cudaError_t launch_combine_backward(const CombineBackwardArgs& a, cudaStream_t stream);
+
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
 

@@ -61,6 +61,7 @@ SIGNATURES = {
     "ep_layout_dispatch": (ctypes.c_int, [_HP, _P, _I32, _P, _P, _P, _P, _SZ, ctypes.c_int, _P, _P, _I32,
                                           _P, _P, _P]),
     "ep_combine": (ctypes.c_int, [_HP, _P, _I32, _P, _P, _P, _P, _P]),
+    "ep_combine_backward": (ctypes.c_int, [_HP, _P, _P, _I32, _P, _P, _P, _P]),
     "ep_read_total_rows": (ctypes.c_int, [_HP, ctypes.POINTER(_I32), _P]),
     "ep_check_error": (ctypes.c_int, [_HP, ctypes.POINTER(ctypes.c_uint32), _P]),
 }
@@ -364,3 +365,32 @@ def combine(y: torch.Tensor, handle: EPHandle, topk_weights: Optional[torch.Tens
     _check(lib().ep_combine(handle.ref, y.data_ptr(), H, _ptr(topk_weights), _ptr(recv_topk_weights),
                             _ptr(out_w), out.data_ptr(), _stream(dev)), "combine")
     return out, out_w
+
+
+def combine_backward(grad_out: torch.Tensor, y: torch.Tensor, handle: EPHandle,
+                     topk_weights: Optional[torch.Tensor] = None, *,
+                     grad_y: Optional[torch.Tensor] = None,
+                     grad_weights: Optional[torch.Tensor] = None):
+    """Backward of combine(y, handle, topk_weights) for the output gradient
+    grad_out [T,H] bf16 -> (grad_y [max_recv_rows,H] bf16, grad_weights [T,k] f32)."""
+    dev = handle.device
+    T, k = handle.num_tokens, handle.num_topk
+    _need(grad_out, "grad_out", (torch.bfloat16,), dev, 2)
+    _need(y, "y", (torch.bfloat16,), dev, 2)
+    H = grad_out.shape[1]
+    if tuple(grad_out.shape) != (T, H) or tuple(y.shape) != (handle.max_recv_rows, H):
+        raise ValueError("grad_out must be [T, hidden] and y [max_recv_rows, hidden]")
+    if topk_weights is not None:
+        _need(topk_weights, "topk_weights", (torch.float32,), dev, 2)
+        if tuple(topk_weights.shape) != (T, k):
+            raise ValueError("topk_weights must be [T, k]")
+    if grad_y is None:
+        grad_y = torch.empty_like(y)
+    if grad_weights is None:
+        grad_weights = torch.empty(T, k, dtype=torch.float32, device=dev)
+    _need(grad_y, "grad_y", (torch.bfloat16,), dev, 2)
+    _need(grad_weights, "grad_weights", (torch.float32,), dev, 2)
+    _check(lib().ep_combine_backward(handle.ref, grad_out.data_ptr(), y.data_ptr(), H, _ptr(topk_weights),
+                                     grad_y.data_ptr(), grad_weights.data_ptr(), _stream(dev)),
+           "combine_backward")
+    return grad_y, grad_weights

@@ -216,6 +216,20 @@ EP_API ep_status ep_combine(const ep_handle* handle, const void* y, int32_t hidd
                             const float* topk_weights, const float* recv_weights_in,
                             float* out_weights, void* out, ep_stream_t stream);
 
+/* Backward of the weighted combine (combine_backward of the DeepEP V2
+ * README, "Interfaces and examples", which runs as a dispatch of the output
+ * gradient; with weights in the forward each row is also scaled):
+ *   grad_y[slot_map[t*k+j], :] = bf16(w[t,j] * grad_out[t, :])   (binary32 product,
+ *                                 one bf16 rounding); padding rows zeroed; rows >= R untouched
+ *   grad_weights[t, j] = sum_h grad_out[t,h] * y[slot_map[t*k+j], h]   (binary32
+ *                                 accumulation, fixed order; 0 for a dropped slot)
+ *   grad_out     [T,H] bf16;  y [max_recv_rows,H] bf16 (the forward's expert outputs)
+ *   topk_weights [T,k] f32, or NULL (every w = 1)
+ *   grad_y       [max_recv_rows,H] bf16 out;  grad_weights [T,k] f32 out.  H % 8 == 0. */
+EP_API ep_status ep_combine_backward(const ep_handle* handle, const void* grad_out, const void* y,
+                                     int32_t hidden, const float* topk_weights, void* grad_y,
+                                     float* grad_weights, ep_stream_t stream);
+
 /* Copies R = offsets[E] to *total_rows on the host.  Synchronises `stream`. */
 EP_API ep_status ep_read_total_rows(const ep_handle* handle, int32_t* total_rows,
                                     ep_stream_t stream);
