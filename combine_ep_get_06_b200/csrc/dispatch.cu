@@ -14,8 +14,9 @@
 //
 // A CTA walks rows grid-stride: token rows [0, T), then padding batches of
 // 32 rows.  Launched with programmatic dependent launch: a CTA waits for
-// the previous grid before reading anything, and lets the next grid start
-// launching once it has issued all its copies.
+// the previous grid before reading what it may have written (directly after
+// the layout, only the routing), and lets the next grid start launching
+// once it has issued all its copies.
 #include "dispatch_device.cuh"
 
 namespace ep {
@@ -30,6 +31,11 @@ constexpr int kPre = 2;  // 32-item slices per warp whose loads are prefetched
 //       [row_bytes] zeros | [scale_pad] zeros | [2][kMaxTopk] int rows
 __host__ __device__ inline size_t smem_bytes(const Geometry& g) {
     return (size_t)3 * g.row_bytes + (size_t)3 * g.scale_pad + 2 * kMaxTopk * sizeof(int);
+}
+
+// Index of the scale of block b of receive row `row` (row- or MN-major).
+__device__ __forceinline__ size_t scale_at(const DispatchArgs& a, int row, int b) {
+    return a.scales_ld > 0 ? (size_t)b * a.scales_ld + row : (size_t)row * (a.H / 128) + b;
 }
 
 template <int kMode>
@@ -61,12 +67,16 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchArgs a) {
         reinterpret_cast<uint4*>(zeros)[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
 
-    // Everything below may read what the layout (the previous grid) wrote.
+    // Right after the layout x is already complete (every layout kernel waits
+    // for the grid before it before letting this one launch), so the first
+    // row's loads can fly while the layout finishes.  Everything the layout
+    // writes is read only after the wait.
+    Item next[kPre];
+    if (a.x_ready) prefetch<kMode>(a, blockIdx.x, geo.ipr, next);
     pdl_wait();
+    if (!a.x_ready) prefetch<kMode>(a, blockIdx.x, geo.ipr, next);
     const int n_pad = ld_cg(a.num_pad_rows);
     const int n_pad_batches = (n_pad + 31) / 32;
-    Item next[kPre];
-    prefetch<kMode>(a, blockIdx.x, geo.ipr, next);
     __syncthreads();
 
     int it = 0;  // token rows handled by this CTA (selects the buffer)
@@ -82,7 +92,7 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchArgs a) {
                         bulk_s2g(rscl + (size_t)row * geo.scale_bytes, zeros + geo.row_bytes, geo.scale_bytes);
                     bulk_commit();
                     if (kFp8Out && !a.bulk_scales)
-                        for (int b = 0; b < B; ++b) a.recv_scales[(size_t)row * B + b] = 0.0f;
+                        for (int b = 0; b < B; ++b) a.recv_scales[scale_at(a, row, b)] = 0.0f;
                 }
             }
             continue;
@@ -127,10 +137,10 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchArgs a) {
             bulk_commit();
         }
         if (kFp8Out && !a.bulk_scales) {
-            // Scale rows not a multiple of 16 bytes: plain stores.
+            // MN-major scales, or rows not a multiple of 16 bytes: plain stores.
             for (int i = tid; i < k * B; i += kThreads) {
                 const int row = rows[i / B];
-                if (row >= 0 && row < a.max_rows) a.recv_scales[(size_t)row * B + i % B] = sb[i % B];
+                if (row >= 0 && row < a.max_rows) a.recv_scales[scale_at(a, row, i % B)] = sb[i % B];
             }
         }
     }

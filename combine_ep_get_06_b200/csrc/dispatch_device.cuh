@@ -1,5 +1,4 @@
-// Per-item work of dispatch, shared by the dispatch kernel and the fused
-// small-batch layout+dispatch kernel.  An item is 16 bytes of one receive
+// Per-item work of the dispatch kernel.  An item is 16 bytes of one receive
 // row: 8 bf16 values (EP_X_BF16), 16 e4m3 values copied (EP_X_FP8), or 16
 // bf16 values quantised to 16 e4m3 bytes (EP_X_BF16_TO_FP8).
 #pragma once

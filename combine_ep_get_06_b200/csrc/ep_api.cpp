@@ -250,6 +250,8 @@ ep_status prepare_dispatch(const ep_handle* h, ep_x_mode mode, const void* x, co
     a->max_rows = h->max_recv_rows;
     a->max_pad_rows = h->num_experts * (h->expert_alignment - 1);
     a->bulk_scales = fp8 && ((H / 128) * 4) % 16 == 0 && aligned(recv_scales, 16);
+    a->x_ready = 0;
+    a->scales_ld = 0;
     return EP_OK;
 }
 
@@ -280,6 +282,24 @@ EP_API ep_status ep_dispatch(const ep_handle* h, ep_x_mode mode, const void* x, 
     return ok();
 }
 
+EP_API ep_status ep_dispatch_mn_scales(const ep_handle* h, ep_x_mode mode, const void* x, const float* x_scales,
+                                       int32_t H, void* recv_x, float* recv_scales_mn, int32_t scales_ld,
+                                       ep_stream_t stream) {
+    ep::DispatchArgs a;
+    ep_status st = prepare_dispatch(h, mode, x, x_scales, H, recv_x, recv_scales_mn, &a);
+    if (st != EP_OK) return st;
+    if (mode == EP_X_BF16) return invalid("MN-major scales need an FP8 mode");
+    if (scales_ld < h->max_recv_rows || scales_ld % 4 != 0)
+        return invalid("scales_ld %d must be >= max_recv_rows (%d) and a multiple of 4", scales_ld,
+                       h->max_recv_rows);
+    if (!aligned(recv_scales_mn, 16)) return invalid("recv_scales_mn must be 16-byte aligned");
+    a.scales_ld = scales_ld;
+    a.bulk_scales = 0;
+    cudaError_t err = ep::launch_dispatch(a, mode, (cudaStream_t)stream);
+    if (err != cudaSuccess) return cuda_failed("dispatch launch", err);
+    return ok();
+}
+
 EP_API ep_status ep_layout_dispatch(ep_handle* h, const void* topk_idx, int32_t idx_is_int64,
                                     const float* topk_weights, int32_t* recv_topk_idx,
                                     float* recv_topk_weights, void* workspace, size_t workspace_bytes,
@@ -292,14 +312,10 @@ EP_API ep_status ep_layout_dispatch(ep_handle* h, const void* topk_idx, int32_t 
     if (st != EP_OK) return st;
     st = prepare_dispatch(h, mode, x, x_scales, H, recv_x, recv_scales, &da);
     if (st != EP_OK) return st;
-    cudaError_t err;
-    if (la.num_chunks == 1 &&
-        ep::layout_dispatch_smem_bytes(mode, H, h->num_experts, h->num_segments) <= ep::kMaxFusedSmem) {
-        err = ep::launch_layout_dispatch(la, da, mode, idx_is_int64 == 1, (cudaStream_t)stream);
-        if (err != cudaSuccess) return cuda_failed("fused layout+dispatch launch", err);
-        return ok();
-    }
-    err = ep::launch_layout(la, idx_is_int64 == 1, (cudaStream_t)stream);
+    // The dispatch launches while the layout runs and loads its x rows before
+    // waiting for it (x_ready); only the routing is read after the wait.
+    da.x_ready = 1;
+    cudaError_t err = ep::launch_layout(la, idx_is_int64 == 1, (cudaStream_t)stream);
     if (err != cudaSuccess) return cuda_failed("layout launch", err);
     err = ep::launch_dispatch(da, mode, (cudaStream_t)stream);
     if (err != cudaSuccess) return cuda_failed("dispatch launch", err);
@@ -380,6 +396,17 @@ EP_API ep_status ep_read_total_rows(const ep_handle* h, int32_t* total_rows, ep_
     if (err == cudaSuccess) err = cudaStreamSynchronize((cudaStream_t)stream);
     if (err != cudaSuccess) return cuda_failed("reading total rows", err);
     *total_rows = v;
+    return ok();
+}
+
+EP_API ep_status ep_read_recv_counts(const ep_handle* h, int32_t* host_counts, ep_stream_t stream) {
+    ep_status st = check_handle(h);
+    if (st != EP_OK) return st;
+    if (host_counts == nullptr) return invalid("host_counts is NULL");
+    cudaError_t err = cudaMemcpyAsync(host_counts, h->recv_counts, sizeof(int32_t) * h->num_experts,
+                                      cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+    if (err == cudaSuccess) err = cudaStreamSynchronize((cudaStream_t)stream);
+    if (err != cudaSuccess) return cuda_failed("reading the per-expert rows", err);
     return ok();
 }
 

@@ -49,6 +49,9 @@ struct DispatchArgs {
     int32_t T, k, H, max_rows;
     int32_t max_pad_rows;  // E*(alignment-1): bound on the padding rows
     int32_t bulk_scales;  // scale rows are a multiple of 16 bytes and recv_scales is 16-byte aligned
+    int32_t x_ready;      // 1: x was complete before the previous grid let this one launch, so it
+                          // may be read before waiting on that grid (only right after the layout)
+    int32_t scales_ld;    // 0: scales row-major [rows][B]; > 0: MN-major [B][scales_ld]
 };
 
 // Shared memory one dispatch CTA needs for this mode and hidden size.
@@ -56,12 +59,6 @@ size_t dispatch_smem_bytes(ep_x_mode mode, int H);
 constexpr size_t kMaxDispatchSmem = 200 * 1024;
 
 cudaError_t launch_dispatch(const DispatchArgs& a, ep_x_mode mode, cudaStream_t stream);
-
-// Fused layout + dispatch for T*k <= kLayoutThreads.
-size_t layout_dispatch_smem_bytes(ep_x_mode mode, int H, int E, int S);
-constexpr size_t kMaxFusedSmem = 220 * 1024;
-cudaError_t launch_layout_dispatch(const LayoutArgs& a, const DispatchArgs& d, ep_x_mode mode,
-                                   bool idx_is_int64, cudaStream_t stream);
 
 struct CombineArgs {
     const void* y;

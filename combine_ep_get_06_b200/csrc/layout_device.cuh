@@ -1,5 +1,4 @@
-// Device building blocks of the layout step, shared by the layout kernels
-// and the fused small-batch layout+dispatch kernel.
+// Device building blocks of the layout kernels.
 //
 // One thread per slot, chunks of <= kThreads slots of whole tokens.  Each
 // slot sets its lane's bit in a per-(warp, expert) word of shared memory

@@ -62,6 +62,8 @@ SIGNATURES = {
                                           _P, _P, _P]),
     "ep_combine": (ctypes.c_int, [_HP, _P, _I32, _P, _P, _P, _P, _P]),
     "ep_combine_backward": (ctypes.c_int, [_HP, _P, _P, _I32, _P, _P, _P, _P]),
+    "ep_dispatch_mn_scales": (ctypes.c_int, [_HP, ctypes.c_int, _P, _P, _I32, _P, _P, _I32, _P]),
+    "ep_read_recv_counts": (ctypes.c_int, [_HP, _P, _P]),
     "ep_read_total_rows": (ctypes.c_int, [_HP, ctypes.POINTER(_I32), _P]),
     "ep_check_error": (ctypes.c_int, [_HP, ctypes.POINTER(ctypes.c_uint32), _P]),
 }
@@ -201,6 +203,13 @@ class EPHandle:
         _check(lib().ep_read_total_rows(self.ref, ctypes.byref(r), _stream(self.device)), "total_rows")
         return r.value
 
+    def recv_counts_host(self) -> list:
+        """Rows of each expert, A(c_e), on the host (synchronises): the
+        pages' num_recv_tokens_per_expert_list."""
+        out = (ctypes.c_int32 * self.num_experts)()
+        _check(lib().ep_read_recv_counts(self.ref, out, _stream(self.device)), "recv_counts_host")
+        return list(out)
+
     def check_error(self) -> int:
         """Reads and clears the device error word; raises EPError if it was set."""
         bits = ctypes.c_uint32(0)
@@ -243,9 +252,10 @@ def get_layout(topk_idx: torch.Tensor, num_experts: int, *, num_segments: int = 
 XType = Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]]
 
 
-def _dispatch_args(x: XType, handle: EPHandle, use_fp8: bool, recv_x, recv_scales):
+def _dispatch_args(x: XType, handle: EPHandle, use_fp8: bool, recv_x, recv_scales, row_scales=True):
     """Checks x and the receive buffers (allocating those not given);
-    returns (mode, x, x_scales, H, recv_x, recv_scales)."""
+    returns (mode, x, x_scales, H, recv_x, recv_scales).  With row_scales
+    False the row-major recv_scales is neither checked nor allocated."""
     dev = handle.device
     rows = handle.max_recv_rows
     x_scales = None
@@ -269,12 +279,13 @@ def _dispatch_args(x: XType, handle: EPHandle, use_fp8: bool, recv_x, recv_scale
     else:
         if recv_x is None:
             recv_x = torch.empty(rows, H, dtype=torch.float8_e4m3fn, device=dev)
-        if recv_scales is None:
-            recv_scales = torch.empty(rows, H // 128, dtype=torch.float32, device=dev)
         _need(recv_x, "recv_x", (torch.float8_e4m3fn, torch.uint8), dev, 2)
-        _need(recv_scales, "recv_scales", (torch.float32,), dev, 2)
-        if tuple(recv_scales.shape) != (rows, H // 128):
-            raise ValueError("recv_scales must be [max_recv_rows, hidden/128]")
+        if row_scales:
+            if recv_scales is None:
+                recv_scales = torch.empty(rows, H // 128, dtype=torch.float32, device=dev)
+            _need(recv_scales, "recv_scales", (torch.float32,), dev, 2)
+            if tuple(recv_scales.shape) != (rows, H // 128):
+                raise ValueError("recv_scales must be [max_recv_rows, hidden/128]")
     if tuple(recv_x.shape) != (rows, H):
         raise ValueError("recv_x must be [max_recv_rows, hidden]")
     return mode, x, x_scales, H, recv_x, recv_scales
@@ -300,8 +311,8 @@ def dispatch(x: XType, topk_idx: Optional[torch.Tensor] = None,
              recv_x: Optional[torch.Tensor] = None, recv_scales: Optional[torch.Tensor] = None,
              recv_topk_idx: Optional[torch.Tensor] = None,
              recv_topk_weights: Optional[torch.Tensor] = None):
-    """MoE dispatch.  With topk_idx: layout and dispatch in one call (one
-    kernel for small batches); returns (recv_x, recv_topk_idx,
+    """MoE dispatch.  With topk_idx: layout and dispatch in one call (the
+    dispatch reads x while the layout runs); returns (recv_x, recv_topk_idx,
     recv_topk_weights, handle).  With only a handle (cached): returns
     (recv_x, None, None, handle)."""
     if topk_idx is None:
@@ -394,3 +405,25 @@ def combine_backward(grad_out: torch.Tensor, y: torch.Tensor, handle: EPHandle,
                                      grad_y.data_ptr(), grad_weights.data_ptr(), _stream(dev)),
            "combine_backward")
     return grad_y, grad_weights
+
+
+def dispatch_mn_scales(x: XType, handle: EPHandle, *, recv_x: Optional[torch.Tensor] = None,
+                       recv_scales_mn: Optional[torch.Tensor] = None, scales_ld: Optional[int] = None):
+    """FP8 dispatch with GEMM-ready scales: recv_scales_mn [H/128, scales_ld]
+    (MN-major, scales_ld = max_recv_rows rounded up to 4 by default).
+    x is bf16 (quantised here) or an (x_fp8, scales) tuple."""
+    dev = handle.device
+    rows = handle.max_recv_rows
+    if scales_ld is None:
+        scales_ld = (rows + 3) // 4 * 4
+    xt = x[0] if isinstance(x, (tuple, list)) else x
+    H = xt.shape[1]
+    if recv_scales_mn is None:
+        recv_scales_mn = torch.empty(H // 128, scales_ld, dtype=torch.float32, device=dev)
+    _need(recv_scales_mn, "recv_scales_mn", (torch.float32,), dev, 2)
+    if tuple(recv_scales_mn.shape) != (H // 128, scales_ld):
+        raise ValueError("recv_scales_mn must be [hidden/128, scales_ld]")
+    mode, x, x_scales, H, recv_x, _ = _dispatch_args(x, handle, True, recv_x, None, row_scales=False)
+    _check(lib().ep_dispatch_mn_scales(handle.ref, mode, x.data_ptr(), _ptr(x_scales), H, recv_x.data_ptr(),
+                                       recv_scales_mn.data_ptr(), scales_ld, _stream(dev)), "dispatch_mn_scales")
+    return recv_x, recv_scales_mn

@@ -191,15 +191,31 @@ EP_API ep_status ep_dispatch(const ep_handle* handle, ep_x_mode mode, const void
  * num_experts, expert_alignment) call of the DeepEP V2 README ("Interfaces
  * and examples"), which routes and sends in one step.  Arguments, results
  * and errors are those of ep_get_layout followed by ep_dispatch with the
- * same handle.  When T*k <= 1024 (a decode step) it runs as ONE kernel in
- * which every CTA computes the small layout itself, instead of two or
- * three launches; otherwise it launches the same kernels as the two calls. */
+ * same handle.  It launches the same kernels, but because it knows that the
+ * dispatch directly follows the layout, the dispatch reads its x rows while
+ * the layout still runs (the two calls cannot assume that). */
 EP_API ep_status ep_layout_dispatch(ep_handle* handle, const void* topk_idx, int32_t idx_is_int64,
                                     const float* topk_weights, int32_t* recv_topk_idx,
                                     float* recv_topk_weights, void* workspace,
                                     size_t workspace_bytes, ep_x_mode mode, const void* x,
                                     const float* x_scales, int32_t hidden, void* recv_x,
                                     float* recv_scales, ep_stream_t stream);
+
+/* Dispatch with the FP8 block scales laid out the way a grouped FP8 GEMM
+ * reads them (DeepEP V2 README, "News": V2 adopts a new GEMM layout;
+ * "Interfaces and examples": the per-expert counts feed the GEMM).  The same
+ * as ep_dispatch in the two FP8 modes, except that the scale of block b of
+ * receive row r goes to recv_scales_mn[b * scales_ld + r] (MN-major: one
+ * column of rows per block).  scales_ld >= max_recv_rows and a multiple of
+ * 4, so that every column starts 16-byte aligned for TMA; entries for rows
+ * >= R and the column tails past max_recv_rows are not written. */
+EP_API ep_status ep_dispatch_mn_scales(const ep_handle* handle, ep_x_mode mode, const void* x,
+                                       const float* x_scales, int32_t hidden, void* recv_x,
+                                       float* recv_scales_mn, int32_t scales_ld, ep_stream_t stream);
+
+/* Copies A(c_e), the rows of each expert (the pages'
+ * num_recv_tokens_per_expert_list), to host_counts[E].  Synchronises `stream`. */
+EP_API ep_status ep_read_recv_counts(const ep_handle* handle, int32_t* host_counts, ep_stream_t stream);
 
 /* Combine (combine_forward; unweighted it is dispatch_backward):
  *   out[t,:] = bf16( sum_j w[t,j] * y[slot_map[t*k+j],:] ) over valid slots,

@@ -155,9 +155,9 @@ def max_bf16_ulp_diff(a_bits: np.ndarray, b_bits: np.ndarray) -> int:
     return int(np.abs(ordered(a_bits) - ordered(b_bits)).max(initial=0))
 
 
-def run_cuda_fused(inp: dict, w: W.Workload, mode: int, *, prequant=None):
-    """layout + dispatch through ep.dispatch(x, topk_idx, ...) (one kernel
-    when T*k <= 1024); returns host arrays like run_cuda (no combine)."""
+def run_cuda_one_call(inp: dict, w: W.Workload, mode: int, *, prequant=None):
+    """layout + dispatch through one ep.dispatch(x, topk_idx, ...) call;
+    returns host arrays like run_cuda (no combine)."""
     T = inp["x"].shape[0]
     idx = torch.from_numpy(inp["topk_idx"]).cuda()
     wts = torch.from_numpy(inp["topk_weights"]).cuda()

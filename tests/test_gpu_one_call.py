@@ -1,6 +1,7 @@
 """The one-call dispatch (layout + dispatch, ep_layout_dispatch) vs the
-oracle: a single fused kernel when T*k <= 1024 slots, the separate kernels
-otherwise.  Bit-exact on every output, guard bytes untouched."""
+oracle.  Here the dispatch reads its x rows before waiting on the layout,
+so these cases cover that ordering, small (one layout CTA) and large (two
+layout kernels).  Bit-exact on every output, guard bytes untouched."""
 
 import numpy as np
 import pytest
@@ -9,7 +10,7 @@ import torch
 import oracle
 import workloads as W
 import combine_ep_get_06_b200 as ep
-from gpu_helpers import assert_parity, run_cuda_fused, run_oracle
+from gpu_helpers import assert_parity, run_cuda_one_call, run_oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -33,16 +34,16 @@ def _random_case(T, k, E, S, align, H, drop, seed, duplicates=False):
 
 
 @pytest.mark.parametrize("name", ["decode", "tiny", "mid"])
-def test_fused_dispatch_on_workloads(name):
+def test_one_call_dispatch_on_workloads(name):
     w = W.WORKLOADS[name]
     inp = W.make_inputs(w, seed=3)
     mode = {"bf16": ep.EP_X_BF16, "fp8_quant": ep.EP_X_BF16_TO_FP8}[w.x_mode]
-    assert_parity(run_cuda_fused(inp, w, mode), run_oracle(inp, w, None, mode), mode)
+    assert_parity(run_cuda_one_call(inp, w, mode), run_oracle(inp, w, None, mode), mode)
 
 
 FUSED = [
     # T, k, E, S, align, H, mode, drop, duplicates
-    (128, 8, 256, 8, 128, 7168, "fp8_quant", 0.1, False),   # padding rows on the fused path
+    (128, 8, 256, 8, 128, 7168, "fp8_quant", 0.1, False),   # padding rows
     (170, 6, 64, 8, 16, 4096, "fp8_quant", 0.05, False),    # k does not divide 32
     (500, 2, 16, 4, 1, 256, "bf16", 0.0, False),            # more tokens than CTAs
     (1024, 1, 7, 7, 3, 128, "fp8_quant", 0.2, False),       # k = 1, 1024 slots
@@ -50,32 +51,32 @@ FUSED = [
     (100, 10, 12, 3, 5, 384, "fp8_quant", 0.3, True),       # duplicate experts, ragged scale rows
     (1, 1, 1, 1, 1, 8, "bf16", 0.0, False),
     (0, 4, 8, 2, 4, 128, "fp8_quant", 0.0, False),          # empty batch
-    (300, 4, 32, 4, 8, 512, "bf16", 0.0, False),            # 1200 slots: separate kernels
+    (300, 4, 32, 4, 8, 512, "bf16", 0.0, False),            # 1200 slots: two layout kernels
 ]
 
 
 @pytest.mark.parametrize("T,k,E,S,align,H,xm,drop,dup", FUSED)
-def test_fused_dispatch_edge_shapes(T, k, E, S, align, H, xm, drop, dup):
-    w = W.Workload("fused", T=T, H=H, E=E, S=S, k=k, align=align, x_mode=xm)
+def test_one_call_dispatch_edge_shapes(T, k, E, S, align, H, xm, drop, dup):
+    w = W.Workload("one_call", T=T, H=H, E=E, S=S, k=k, align=align, x_mode=xm)
     inp = _random_case(T, k, E, S, align, H, drop, seed=T + 7 * k, duplicates=dup)
     mode = {"bf16": ep.EP_X_BF16, "fp8_quant": ep.EP_X_BF16_TO_FP8}[xm]
-    assert_parity(run_cuda_fused(inp, w, mode), run_oracle(inp, w, None, mode), mode)
+    assert_parity(run_cuda_one_call(inp, w, mode), run_oracle(inp, w, None, mode), mode)
 
 
-def test_fused_dispatch_prequantised_tuple():
+def test_one_call_dispatch_prequantised_tuple():
     w = W.Workload("pq", T=96, H=1024, E=32, S=4, k=8, align=4, x_mode="fp8_quant")
     inp = _random_case(96, 8, 32, 4, 4, 1024, 0.1, seed=11)
     pq = W.make_prequant(96, 1024, seed=11)
-    g = run_cuda_fused(inp, w, ep.EP_X_FP8, prequant=pq)
+    g = run_cuda_one_call(inp, w, ep.EP_X_FP8, prequant=pq)
     assert_parity(g, run_oracle(inp, w, None, oracle.X_FP8_PREQUANT, prequant=pq), oracle.X_FP8_PREQUANT)
 
 
-def test_fused_dispatch_flags_bad_indices():
+def test_one_call_dispatch_flags_bad_indices():
     w = W.Workload("bad", T=64, H=256, E=16, S=4, k=4, align=2, x_mode="fp8_quant")
     inp = _random_case(64, 4, 16, 4, 2, 256, 0.0, seed=5)
     inp["topk_idx"][3, 2] = 99
     inp["topk_idx"][40, 0] = -5
-    g = run_cuda_fused(inp, w, ep.EP_X_BF16_TO_FP8)
+    g = run_cuda_one_call(inp, w, ep.EP_X_BF16_TO_FP8)
     o = run_oracle(inp, w, None, oracle.X_BF16_QUANT_FP8)
     assert_parity(g, o, oracle.X_BF16_QUANT_FP8)
     with pytest.raises(ep.EPError, match="topk_idx"):
