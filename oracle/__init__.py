@@ -20,7 +20,7 @@ from . import build as _build
 
 _lib = None
 
-X_BF16, X_FP8_PREQUANT, X_BF16_QUANT_FP8 = 0, 1, 2
+X_BF16, X_FP8_PREQUANT, X_BF16_QUANT_FP8, X_BF16_QUANT_NVFP4 = 0, 1, 2, 3
 
 
 def lib():
@@ -46,6 +46,14 @@ def lib():
         L.oracle_e4m3_encode_n.restype = None
         L.oracle_quantize_rows.argtypes = [i64, i32, P, P, P]
         L.oracle_quantize_rows.restype = None
+        L.oracle_e2m1_encode.argtypes = [ctypes.c_float]
+        L.oracle_e2m1_encode.restype = ctypes.c_uint8
+        L.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
+        L.oracle_e2m1_decode.restype = ctypes.c_float
+        L.oracle_e2m1_encode_n.argtypes = [P, P, i64]
+        L.oracle_e2m1_encode_n.restype = None
+        L.oracle_nvfp4_rows.argtypes = [i64, i32, P, P, P]
+        L.oracle_nvfp4_rows.restype = None
         L.oracle_max_recv_rows.argtypes = [i32, i32, i32, i32]
         L.oracle_max_recv_rows.restype = i32
         L.oracle_layout.argtypes = [i32, i32, i32, i32, i32, P, P, i32, P, P, P, P, P, P, P]
@@ -107,6 +115,30 @@ def quantize_rows(x_bf16: np.ndarray):
     return q, s
 
 
+def e2m1_encode(v: np.ndarray) -> np.ndarray:
+    v = _c(v, np.float32)
+    out = np.empty(v.shape, dtype=np.uint8)
+    lib().oracle_e2m1_encode_n(_p(v), _p(out), v.size)
+    return out
+
+
+def e2m1_decode(c: np.ndarray) -> np.ndarray:
+    c = _c(c, np.uint8)
+    L = lib()
+    table = np.array([L.oracle_e2m1_decode(i) for i in range(16)], dtype=np.float32)
+    return table[c & 0xF]
+
+
+def nvfp4_rows(x_bf16: np.ndarray):
+    """bf16 bits [rows, H] -> (packed e2m1 [rows, H/2] uint8, e4m3 scales [rows, H/16] uint8)."""
+    x = _c(x_bf16, np.uint16)
+    rows, H = x.shape
+    q = np.empty((rows, H // 2), dtype=np.uint8)
+    s = np.empty((rows, H // 16), dtype=np.uint8)
+    lib().oracle_nvfp4_rows(rows, H, _p(x), _p(q), _p(s))
+    return q, s
+
+
 # ------------------------------------------------------------------- layout
 
 def max_recv_rows(T: int, k: int, E: int, align: int) -> int:
@@ -149,6 +181,10 @@ def dispatch(lay: dict, x: np.ndarray, mode: int, x_scales=None):
         x = _c(x, np.uint16)
         recv = np.full((cap, x.shape[1]), UNWRITTEN * 0x0101, np.uint16)
         scales = None
+    elif mode == X_BF16_QUANT_NVFP4:
+        x = _c(x, np.uint16)
+        recv = np.full((cap, x.shape[1] // 2), UNWRITTEN, np.uint8)
+        scales = np.full((cap, x.shape[1] // 16), UNWRITTEN, np.uint8)
     else:
         x = _c(x, np.uint8 if mode == X_FP8_PREQUANT else np.uint16)
         recv = np.full((cap, x.shape[1]), UNWRITTEN, np.uint8)

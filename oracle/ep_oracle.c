@@ -47,6 +47,13 @@
  *     q = e4m3(x * inv) rounded to nearest-even with saturation to +-448;
  *   - combine: acc = +0.0f, then for j = 0..k-1 over valid slots
  *     acc = fmaf(w[t,j], y[row], acc), and one bf16 rounding at the end;
+ *   - NVFP4 dispatch (the Hybrid-EP branch of the DeepEP V2 README lists the
+ *     NVFP4 data type; nothing more is stated): E2M1 values in 1x16 blocks,
+ *     one E4M3 scale per block, no per-tensor scale: amax = max |x| floored
+ *     at 6 * 2^-9, scale = e4m3(amax / 6) (nearest-even, saturating),
+ *     inv = 1 / scale (one IEEE division), q = e2m1(x * inv) rounded to
+ *     nearest-even and saturating at +-6; two codes per byte, the even
+ *     element in the low nibble;
  *   - combine backward: grad_y[row] = bf16(w * g) with the product taken in
  *     binary32 (one multiply, one bf16 rounding); padding rows of grad_y are
  *     zero; grad_w is the exact dot product, accumulated here in binary64
@@ -157,6 +164,66 @@ EXPORT void oracle_quantize_rows(int64_t rows, int32_t H, const uint16_t* x, uin
                            scales + r * nb + b);
 }
 
+/* ---------------------------------------------------- NVFP4 (E2M1, 1x16) */
+
+/* 4-bit float E2M1: sign, 2 exponent bits (bias 1), 1 mantissa bit, no
+ * infinities or NaN.  Magnitudes: exponent field 0 holds 0 and 0.5 (m * 0.5);
+ * field f >= 1 holds (1 + m/2) * 2^(f-1): 1, 1.5, 2, 3, 4, 6.  Encoding:
+ * nearest, ties to even mantissa, saturating at 6. */
+EXPORT uint8_t oracle_e2m1_encode(float v) {
+    uint8_t sign = signbit(v) ? 0x8 : 0x0;
+    float a = fabsf(v);
+    if (isnan(v)) return sign | 0x7;          /* unspecified; never produced by finite inputs */
+    if (a >= 6.0f) return sign | 0x7;
+    float quantum;                            /* spacing of the grid at a's magnitude */
+    int field;
+    if (a < 2.0f) { quantum = 0.5f; field = 0; }
+    else if (a < 4.0f) { quantum = 1.0f; field = 2; }
+    else { quantum = 2.0f; field = 3; }
+    int n = (int)rintf(a / quantum);          /* exact scaling, nearest-even */
+    if (field == 0) {                         /* [0, 2): 0, 0.5, 1, 1.5 -> codes 0..3; 2 -> code 4 */
+        return sign | (uint8_t)n;
+    }
+    if (field == 2) {                         /* [2, 4): n in {2, 3, 4}: 2 -> 0x4, 3 -> 0x5, 4 -> 0x6 */
+        return sign | (uint8_t)(n + 2);
+    }
+    return sign | (uint8_t)(n == 2 ? 0x6 : 0x7); /* [4, 6): n in {2, 3}: 4 -> 0x6, 6 -> 0x7 */
+}
+
+EXPORT float oracle_e2m1_decode(uint8_t c) {
+    static const float mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+    return (c & 0x8) ? -mag[c & 7] : mag[c & 7];
+}
+
+EXPORT void oracle_e2m1_encode_n(const float* v, uint8_t* out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_e2m1_encode(v[i]);
+}
+
+#define FP4BLOCK 16
+static const float E2M1_MAX = 6.0f;
+static const float FP4_AMAX_FLOOR = 6.0f / 512.0f;   /* 6 * 2^-9: smallest e4m3 scale */
+
+/* One 1x16 block of bf16 -> 8 bytes of E2M1 pairs and one E4M3 scale byte. */
+static void nvfp4_block(const uint16_t* x, uint8_t* q, uint8_t* scale) {
+    float amax = 0.0f;
+    for (int i = 0; i < FP4BLOCK; ++i) amax = fmaxf(amax, fabsf(oracle_bf16_to_f32(x[i])));
+    if (amax < FP4_AMAX_FLOOR) amax = FP4_AMAX_FLOOR;
+    *scale = oracle_e4m3_encode(amax / E2M1_MAX);
+    float inv = 1.0f / oracle_e4m3_decode(*scale);
+    for (int i = 0; i < FP4BLOCK; i += 2)
+        q[i / 2] = (uint8_t)(oracle_e2m1_encode(oracle_bf16_to_f32(x[i]) * inv) |
+                             (oracle_e2m1_encode(oracle_bf16_to_f32(x[i + 1]) * inv) << 4));
+}
+
+/* A [rows, H] bf16 matrix -> packed E2M1 [rows, H/2] and scales [rows, H/16]. */
+EXPORT void oracle_nvfp4_rows(int64_t rows, int32_t H, const uint16_t* x, uint8_t* q, uint8_t* scales) {
+    int32_t nb = H / FP4BLOCK;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int32_t b = 0; b < nb; ++b)
+            nvfp4_block(x + r * H + (int64_t)b * FP4BLOCK, q + r * (H / 2) + (int64_t)b * (FP4BLOCK / 2),
+                        scales + r * nb + b);
+}
+
 /* ---------------------------------------------------------------- layout */
 
 EXPORT int32_t oracle_max_recv_rows(int32_t T, int32_t k, int32_t E, int32_t align) {
@@ -239,21 +306,23 @@ EXPORT uint32_t oracle_layout(int32_t T, int32_t k, int32_t E, int32_t S, int32_
 
 /* -------------------------------------------------------------- dispatch */
 
-enum { ORACLE_X_BF16 = 0, ORACLE_X_FP8_PREQUANT = 1, ORACLE_X_BF16_QUANT_FP8 = 2 };
+enum { ORACLE_X_BF16 = 0, ORACLE_X_FP8_PREQUANT = 1, ORACLE_X_BF16_QUANT_FP8 = 2, ORACLE_X_BF16_QUANT_NVFP4 = 3 };
 
 /* Copies token t's row into row slot_map[t*k+j] for every valid j, and zeroes
  * the padding rows (rows r < R with recv_src[r] < 0).
  *   mode 0: x bf16 [T,H]                  -> recv_x bf16 [*,H]
- *   mode 1: x e4m3 [T,H], x_scales [T,H/128] -> recv_x e4m3, recv_scales
- *   mode 2: x bf16 [T,H], quantised here   -> recv_x e4m3, recv_scales   */
+ *   mode 1: x e4m3 [T,H], x_scales [T,H/128] -> recv_x e4m3, recv_scales f32
+ *   mode 2: x bf16 [T,H], quantised here   -> recv_x e4m3, recv_scales f32 [*,H/128]
+ *   mode 3: x bf16 [T,H], NVFP4 here       -> recv_x [*,H/2] bytes, recv_scales e4m3 bytes [*,H/16] */
 EXPORT void oracle_dispatch(int32_t mode, int32_t T, int32_t k, int32_t H, int32_t R,
                             const int32_t* slot_map, const int32_t* recv_src, const void* x,
-                            const float* x_scales, void* recv_x, float* recv_scales) {
-    int32_t nb = H / QBLOCK;
-    size_t elem = (mode == ORACLE_X_BF16) ? 2 : 1;
-    size_t row_bytes = (size_t)H * elem;
+                            const float* x_scales, void* recv_x, void* recv_scales) {
+    const int fp4 = mode == ORACLE_X_BF16_QUANT_NVFP4;
+    int32_t nb = fp4 ? H / FP4BLOCK : H / QBLOCK;
+    size_t row_bytes = mode == ORACLE_X_BF16 ? (size_t)H * 2 : fp4 ? (size_t)H / 2 : (size_t)H;
+    size_t scale_bytes = fp4 ? (size_t)nb : sizeof(float) * (size_t)nb;
     uint8_t* qrow = (uint8_t*)malloc((size_t)H);
-    float* srow = (float*)malloc(sizeof(float) * (nb > 0 ? nb : 1));
+    uint8_t* srow = (uint8_t*)malloc(scale_bytes > 0 ? scale_bytes : 1);
 
     for (int32_t t = 0; t < T; ++t) {
         const uint8_t* src;
@@ -263,26 +332,31 @@ EXPORT void oracle_dispatch(int32_t mode, int32_t T, int32_t k, int32_t H, int32
         } else if (mode == ORACLE_X_FP8_PREQUANT) {
             src = (const uint8_t*)x + (size_t)t * row_bytes;
             src_scales = x_scales + (size_t)t * nb;
+        } else if (fp4) {
+            const uint16_t* xt = (const uint16_t*)x + (size_t)t * H;
+            for (int32_t b = 0; b < nb; ++b)
+                nvfp4_block(xt + b * FP4BLOCK, qrow + b * (FP4BLOCK / 2), srow + b);
+            src = qrow;
+            src_scales = (const float*)srow;
         } else {
             const uint16_t* xt = (const uint16_t*)x + (size_t)t * H;
             for (int32_t b = 0; b < nb; ++b)
-                quantize_block(xt + b * QBLOCK, qrow + b * QBLOCK, srow + b);
+                quantize_block(xt + b * QBLOCK, qrow + b * QBLOCK, (float*)srow + b);
             src = qrow;
-            src_scales = srow;
+            src_scales = (const float*)srow;
         }
         for (int32_t j = 0; j < k; ++j) {
             int32_t row = slot_map[(int64_t)t * k + j];
             if (row < 0) continue;
             memcpy((uint8_t*)recv_x + (size_t)row * row_bytes, src, row_bytes);
             if (mode != ORACLE_X_BF16)
-                memcpy(recv_scales + (size_t)row * nb, src_scales, sizeof(float) * nb);
+                memcpy((uint8_t*)recv_scales + (size_t)row * scale_bytes, src_scales, scale_bytes);
         }
     }
     for (int32_t row = 0; row < R; ++row) {
         if (recv_src[row] >= 0) continue;
         memset((uint8_t*)recv_x + (size_t)row * row_bytes, 0, row_bytes);
-        if (mode != ORACLE_X_BF16)
-            for (int32_t b = 0; b < nb; ++b) recv_scales[(size_t)row * nb + b] = 0.0f;
+        if (mode != ORACLE_X_BF16) memset((uint8_t*)recv_scales + (size_t)row * scale_bytes, 0, scale_bytes);
     }
     free(srow);
     free(qrow);

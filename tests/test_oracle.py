@@ -153,6 +153,68 @@ def test_e4m3_decoder_matches_torch():
     assert np.array_equal(ours[~nan], ref[~nan])
 
 
+def e2m1_brute(v: np.ndarray) -> np.ndarray:
+    """Nearest of the 8 E2M1 magnitudes by exhaustive search (ties: even
+    mantissa = even code), saturating at 6, sign reapplied."""
+    mags = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    a = np.minimum(np.abs(v.astype(np.float64)), 6.0)
+    d = np.abs(a[:, None] - mags[None, :])
+    cand = d == d.min(axis=1, keepdims=True)
+    even = (np.arange(8) & 1) == 0
+    pick = np.where((cand & even).any(axis=1), np.argmax(cand & even, axis=1), np.argmax(cand, axis=1))
+    return np.where(np.signbit(v.astype(np.float32)), pick | 8, pick).astype(np.uint8)
+
+
+def test_e2m1_hand_derived_codes(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "e2m1_codes.json")))
+    vals = np.array([float(v) for v in g["values"]], dtype=np.float32)
+    assert np.array_equal(oracle.e2m1_encode(vals), np.array(g["codes"], dtype=np.uint8))
+
+
+def test_e2m1_encoder_matches_brute_force_search():
+    mags = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    pts = np.concatenate([mags, (mags[:-1] + mags[1:]) / 2, [6.5, 7.0, 100.0]]).astype(np.float32)
+    u = pts.view(np.uint32).astype(np.int64)
+    near = (u[:, None] + np.arange(-3, 4)[None, :]).reshape(-1)
+    near = near[near >= 0].astype(np.uint32).view(np.float32)
+    rng = np.random.default_rng(31)
+    v = np.concatenate([near, rng.uniform(0, 8, 100_000).astype(np.float32), [0.0]])
+    v = np.concatenate([v, -v])
+    assert np.array_equal(oracle.e2m1_encode(v), e2m1_brute(v))
+    assert np.array_equal(oracle.e2m1_decode(np.arange(16, dtype=np.uint8)),
+                          np.concatenate([mags, -mags]).astype(np.float32))
+
+
+def test_nvfp4_block_invariants():
+    rng = np.random.default_rng(37)
+    H = 512
+    x = rng.standard_normal((40, H)) * (10.0 ** rng.uniform(-1.5, 2.5, size=(40, H // 16))).repeat(16, axis=1)
+    x[3, 16:32] = 0.0                                        # zero block -> smallest scale, zero codes
+    x[4, 0:16] = 0.0
+    x[4, 0], x[4, 1] = 5.0, 0.5                              # nibble order: even element in the low nibble
+    xb = bf16_bits_of(x)
+    xf = f32_of_bf16(xb).reshape(40, H // 16, 16).astype(np.float64)
+    q, s = oracle.nvfp4_rows(xb)
+    codes = np.stack([q & 0xF, q >> 4], axis=-1).reshape(40, H // 16, 16)
+    sdec = oracle.e4m3_decode(s).astype(np.float64)
+    amax = np.maximum(np.abs(xf).max(axis=2), 6.0 / 512)
+    # the scale is the e4m3 rounding of amax/6: within half an e4m3 spacing, codes 0x01..0x7E
+    assert np.all((s >= 1) & (s <= 0x7E))
+    assert np.all(np.abs(sdec - amax / 6) <= 2.0 ** (np.floor(np.log2(np.maximum(amax / 6, 2.0 ** -6))) - 4) + 1e-12)
+    # the largest element of every non-zero block lands on +-6
+    am = np.abs(xf).argmax(axis=2)
+    top = np.take_along_axis(codes, am[..., None], axis=2)[..., 0]
+    nz = np.abs(xf).max(axis=2) > 0
+    assert np.all((top[nz] & 7) == 7)
+    # every code is the nearest E2M1 value (brute force) to x * (1/scale) in
+    # binary32, saturating at 6
+    inv = (np.float32(1.0) / sdec.astype(np.float32))[..., None]
+    t = (xf.astype(np.float32) * inv).astype(np.float32)
+    assert np.array_equal(codes.reshape(-1), e2m1_brute(t.reshape(-1)))
+    assert np.all(codes[3, 1] == 0) and s[3, 1] == 0x01
+    assert q[4, 0] & 0xF == 7 and q[4, 0] >> 4 == codes[4, 0, 1]    # x[0] (5.0, the amax) in the low nibble
+
+
 # ---------------------------------------------------------- quantisation
 
 def test_quantize_hand_example():
@@ -321,6 +383,12 @@ def test_dispatch_rows_are_the_source_tokens(name):
     recv, _ = oracle.dispatch(lay, inp["x"], oracle.X_BF16)
     assert np.array_equal(recv[sm[valid]], inp["x"][src_tok])           # numpy gather
     assert np.all(recv[pad] == 0)
+    if w.H % 16 == 0:
+        q4, s4 = oracle.nvfp4_rows(inp["x"])
+        rq, rs = oracle.dispatch(lay, inp["x"], oracle.X_BF16_QUANT_NVFP4)
+        assert np.array_equal(rq[sm[valid]], q4[src_tok]) and np.array_equal(rs[sm[valid]], s4[src_tok])
+        assert np.all(rq[pad] == 0) and np.all(rs[pad] == 0)
+        assert np.all(rq[R:] == oracle.UNWRITTEN) and np.all(rs[R:] == oracle.UNWRITTEN)
     if w.H % 128 == 0:
         q, s = oracle.quantize_rows(inp["x"])
         rq, rs = oracle.dispatch(lay, inp["x"], oracle.X_BF16_QUANT_FP8)

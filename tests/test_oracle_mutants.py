@@ -39,8 +39,8 @@ MUTANTS = {
     "row weight from wrong slot": ("recv_topk_weights[row] = topk_weights ? topk_weights[s] : 0.0f;",
                                    "recv_topk_weights[row] = topk_weights ? topk_weights[s - s % k] : 0.0f;"),
     "padding not zeroed": ("memset((uint8_t*)recv_x + (size_t)row * row_bytes, 0, row_bytes);", ""),
-    "scales go to the token's row": ("memcpy(recv_scales + (size_t)row * nb, src_scales, sizeof(float) * nb);",
-                                     "memcpy(recv_scales + (size_t)t * nb, src_scales, sizeof(float) * nb);"),
+    "scales go to the token's row": ("memcpy((uint8_t*)recv_scales + (size_t)row * scale_bytes, src_scales, scale_bytes);",
+                                     "memcpy((uint8_t*)recv_scales + (size_t)t * scale_bytes, src_scales, scale_bytes);"),
     "combine sums in reverse order": ("            for (int32_t j = 0; j < k; ++j) {\n                if (sm[j] < 0) continue;",
                                       "            for (int32_t j = k - 1; j >= 0; --j) {\n                if (sm[j] < 0) continue;"),
     "combine weight of wrong slot": ("float w = weights ? weights[(int64_t)t * k + j] : 1.0f;",
@@ -55,6 +55,11 @@ MUTANTS = {
                                               "dot += (double)gv * (double)oracle_bf16_to_f32(y[(size_t)t * H + h]);"),
     "backward padding not zeroed": ("if (recv_src[row] < 0) memset(grad_y + (size_t)row * H, 0, sizeof(uint16_t) * H);",
                                     "if (recv_src[row] < 0) {}"),
+    "e2m1 ties away from even": ("int n = (int)rintf(a / quantum);", "int n = (int)floorf(a / quantum + 0.5f);"),
+    "nvfp4 nibbles swapped": ("q[i / 2] = (uint8_t)(oracle_e2m1_encode(oracle_bf16_to_f32(x[i]) * inv) |\n                             (oracle_e2m1_encode(oracle_bf16_to_f32(x[i + 1]) * inv) << 4));",
+                              "q[i / 2] = (uint8_t)(oracle_e2m1_encode(oracle_bf16_to_f32(x[i + 1]) * inv) |\n                             (oracle_e2m1_encode(oracle_bf16_to_f32(x[i]) * inv) << 4));"),
+    "nvfp4 scale from amax / 4": ("*scale = oracle_e4m3_encode(amax / E2M1_MAX);", "*scale = oracle_e4m3_encode(amax / 4.0f);"),
+    "nvfp4 divides by the unrounded scale": ("float inv = 1.0f / oracle_e4m3_decode(*scale);", "float inv = E2M1_MAX / amax;"),
     "weight gather ignores the slot map": ("(sm[j] >= 0 && recv_weights_in) ? recv_weights_in[sm[j]] : 0.0f;",
                                            "(sm[j] >= 0 && recv_weights_in) ? recv_weights_in[j] : 0.0f;"),
 }
