@@ -324,6 +324,26 @@ def run_ours(args, rank, world, dev):
                                      "gbs": round(nbytes["dispatch"] / (mn_ms * 1e-3) / 1e9, 1),
                                      "frac_of_peak": round(nbytes["dispatch"] / (mn_ms * 1e-3) / 1e9 / peak, 4)}
 
+    # NVFP4 dispatch (E2M1 codes, one e4m3 scale per 1x16 block), same workload
+    if H % 32 == 0:
+        nv_x = torch.empty(rows, H // 2, dtype=torch.uint8, device=dev)
+        nv_s = torch.empty(rows, H // 16, dtype=torch.uint8, device=dev)
+        nv = lambda: ep.dispatch_with_handle(x, handle, use_nvfp4=True, recv_x=nv_x, recv_scales=nv_s)
+        for _ in range(3):
+            nv()
+        n0, n1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_n = max(3, min(50, K))
+        n0.record(stream)
+        for _ in range(n_n):
+            nv()
+        n1.record(stream)
+        torch.cuda.synchronize(dev)
+        nv_ms = n0.elapsed_time(n1) / n_n
+        nv_bytes = T * H * 2 + T * k * 4 + (V + P) * (H // 2 + H // 16)
+        res["dispatch_nvfp4"] = {"us": round(nv_ms * 1e3, 2), "bytes": nv_bytes,
+                                 "gbs": round(nv_bytes / (nv_ms * 1e-3) / 1e9, 1),
+                                 "frac_of_peak": round(nv_bytes / (nv_ms * 1e-3) / 1e9 / peak, 4)}
+
     # the backward of the weighted combine (training), same workload
     gy = torch.empty(rows, H, dtype=torch.bfloat16, device=dev)
     gw = torch.empty(T, k, dtype=torch.float32, device=dev)

@@ -33,9 +33,17 @@ __host__ __device__ inline size_t smem_bytes(const Geometry& g) {
     return (size_t)3 * g.row_bytes + (size_t)3 * g.scale_pad + 2 * kMaxTopk * sizeof(int);
 }
 
-// Index of the scale of block b of receive row `row` (row- or MN-major).
-__device__ __forceinline__ size_t scale_at(const DispatchArgs& a, int row, int b) {
-    return a.scales_ld > 0 ? (size_t)b * a.scales_ld + row : (size_t)row * (a.H / 128) + b;
+// Stores the scale of block b of receive row `row` (f32 row- or MN-major,
+// or an e4m3 byte for NVFP4), taken from the row's scale buffer sb.
+template <int kMode>
+__device__ __forceinline__ void store_scale(const DispatchArgs& a, int row, int b, const float* sb, bool zero) {
+    if (kMode == EP_X_BF16_TO_NVFP4) {
+        reinterpret_cast<unsigned char*>(a.recv_scales)[(size_t)row * (a.H / 16) + b] =
+            zero ? 0 : reinterpret_cast<const unsigned char*>(sb)[b];
+    } else {
+        const size_t at = a.scales_ld > 0 ? (size_t)b * a.scales_ld + row : (size_t)row * (a.H / 128) + b;
+        reinterpret_cast<float*>(a.recv_scales)[at] = zero ? 0.0f : sb[b];
+    }
 }
 
 template <int kMode>
@@ -59,7 +67,8 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchArgs a) {
     int* rows_s = (int*)(zeros + geo.row_bytes + geo.scale_pad);   // [2][kMaxTopk]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int T = a.T, k = a.k, B = a.H / 128;
+    const int T = a.T, k = a.k;
+    const int B = kMode == EP_X_BF16_TO_NVFP4 ? a.H / 16 : a.H / 128;  // scales per row
     char* const recv = (char*)a.recv_x;
     char* const rscl = (char*)a.recv_scales;
 
@@ -92,7 +101,7 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchArgs a) {
                         bulk_s2g(rscl + (size_t)row * geo.scale_bytes, zeros + geo.row_bytes, geo.scale_bytes);
                     bulk_commit();
                     if (kFp8Out && !a.bulk_scales)
-                        for (int b = 0; b < B; ++b) a.recv_scales[scale_at(a, row, b)] = 0.0f;
+                        for (int b = 0; b < B; ++b) store_scale<kMode>(a, row, b, nullptr, true);
                 }
             }
             continue;
@@ -140,7 +149,7 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchArgs a) {
             // MN-major scales, or rows not a multiple of 16 bytes: plain stores.
             for (int i = tid; i < k * B; i += kThreads) {
                 const int row = rows[i / B];
-                if (row >= 0 && row < a.max_rows) a.recv_scales[scale_at(a, row, i % B)] = sb[i % B];
+                if (row >= 0 && row < a.max_rows) store_scale<kMode>(a, row, i % B, sb, false);
             }
         }
     }
@@ -189,6 +198,7 @@ cudaError_t launch_dispatch(const DispatchArgs& a, ep_x_mode mode, cudaStream_t 
         case EP_X_BF16: return launch_t<EP_X_BF16>(a, stream);
         case EP_X_FP8: return launch_t<EP_X_FP8>(a, stream);
         case EP_X_BF16_TO_FP8: return launch_t<EP_X_BF16_TO_FP8>(a, stream);
+        case EP_X_BF16_TO_NVFP4: return launch_t<EP_X_BF16_TO_NVFP4>(a, stream);
     }
     return cudaErrorInvalidValue;
 }

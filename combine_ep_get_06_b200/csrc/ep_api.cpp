@@ -221,17 +221,21 @@ ep_status prepare_layout(ep_handle* h, const void* topk_idx, int32_t idx_is_int6
 
 // Checks the dispatch arguments and fills a.
 ep_status prepare_dispatch(const ep_handle* h, ep_x_mode mode, const void* x, const float* x_scales, int32_t H,
-                           void* recv_x, float* recv_scales, ep::DispatchArgs* a) {
+                           void* recv_x, void* recv_scales, ep::DispatchArgs* a) {
     ep_status st = check_handle(h);
     if (st != EP_OK) return st;
-    if (mode != EP_X_BF16 && mode != EP_X_FP8 && mode != EP_X_BF16_TO_FP8) return invalid("unknown x mode %d", (int)mode);
-    const bool fp8 = mode != EP_X_BF16;
-    if (H < 1 || H % (fp8 ? 128 : 8) != 0)
-        return invalid("hidden %d must be a positive multiple of %d in this mode", H, fp8 ? 128 : 8);
+    if (mode != EP_X_BF16 && mode != EP_X_FP8 && mode != EP_X_BF16_TO_FP8 && mode != EP_X_BF16_TO_NVFP4)
+        return invalid("unknown x mode %d", (int)mode);
+    const bool nvfp4 = mode == EP_X_BF16_TO_NVFP4;
+    const bool fp8 = mode == EP_X_FP8 || mode == EP_X_BF16_TO_FP8;
+    const int hmul = nvfp4 ? 32 : fp8 ? 128 : 8;
+    if (H < 1 || H % hmul != 0)
+        return invalid("hidden %d must be a positive multiple of %d in this mode", H, hmul);
     if (h->num_tokens > 0 && (x == nullptr || !aligned(x, 16))) return invalid("x must be non-NULL and 16-byte aligned");
     if (recv_x == nullptr || !aligned(recv_x, 16)) return invalid("recv_x must be non-NULL and 16-byte aligned");
     if (fp8 && (recv_scales == nullptr || !aligned(recv_scales, 4)))
         return invalid("recv_scales must be non-NULL and 4-byte aligned in the FP8 modes");
+    if (nvfp4 && recv_scales == nullptr) return invalid("recv_scales must be non-NULL in the NVFP4 mode");
     if (mode == EP_X_FP8 && h->num_tokens > 0 && (x_scales == nullptr || !aligned(x_scales, 4)))
         return invalid("x_scales must be non-NULL and 4-byte aligned for pre-quantised x");
     if (ep::dispatch_smem_bytes(mode, H) > ep::kMaxDispatchSmem)
@@ -249,7 +253,8 @@ ep_status prepare_dispatch(const ep_handle* h, ep_x_mode mode, const void* x, co
     a->H = H;
     a->max_rows = h->max_recv_rows;
     a->max_pad_rows = h->num_experts * (h->expert_alignment - 1);
-    a->bulk_scales = fp8 && ((H / 128) * 4) % 16 == 0 && aligned(recv_scales, 16);
+    a->bulk_scales = (fp8 && ((H / 128) * 4) % 16 == 0 && aligned(recv_scales, 16)) ||
+                     (nvfp4 && (H / 16) % 16 == 0 && aligned(recv_scales, 16));
     a->x_ready = 0;
     a->scales_ld = 0;
     return EP_OK;
@@ -273,7 +278,7 @@ EP_API ep_status ep_get_layout(ep_handle* h, const void* topk_idx, int32_t idx_i
 }
 
 EP_API ep_status ep_dispatch(const ep_handle* h, ep_x_mode mode, const void* x, const float* x_scales,
-                             int32_t H, void* recv_x, float* recv_scales, ep_stream_t stream) {
+                             int32_t H, void* recv_x, void* recv_scales, ep_stream_t stream) {
     ep::DispatchArgs a;
     ep_status st = prepare_dispatch(h, mode, x, x_scales, H, recv_x, recv_scales, &a);
     if (st != EP_OK) return st;
@@ -288,7 +293,7 @@ EP_API ep_status ep_dispatch_mn_scales(const ep_handle* h, ep_x_mode mode, const
     ep::DispatchArgs a;
     ep_status st = prepare_dispatch(h, mode, x, x_scales, H, recv_x, recv_scales_mn, &a);
     if (st != EP_OK) return st;
-    if (mode == EP_X_BF16) return invalid("MN-major scales need an FP8 mode");
+    if (mode != EP_X_FP8 && mode != EP_X_BF16_TO_FP8) return invalid("MN-major scales need an FP8 mode");
     if (scales_ld < h->max_recv_rows || scales_ld % 4 != 0)
         return invalid("scales_ld %d must be >= max_recv_rows (%d) and a multiple of 4", scales_ld,
                        h->max_recv_rows);
@@ -304,7 +309,7 @@ EP_API ep_status ep_layout_dispatch(ep_handle* h, const void* topk_idx, int32_t 
                                     const float* topk_weights, int32_t* recv_topk_idx,
                                     float* recv_topk_weights, void* workspace, size_t workspace_bytes,
                                     ep_x_mode mode, const void* x, const float* x_scales, int32_t H,
-                                    void* recv_x, float* recv_scales, ep_stream_t stream) {
+                                    void* recv_x, void* recv_scales, ep_stream_t stream) {
     ep::LayoutArgs la;
     ep::DispatchArgs da;
     ep_status st = prepare_layout(h, topk_idx, idx_is_int64, topk_weights, recv_topk_idx, recv_topk_weights,

@@ -41,7 +41,7 @@ struct DispatchArgs {
     const void* x;
     const float* x_scales;
     void* recv_x;
-    float* recv_scales;
+    void* recv_scales;    // f32 (FP8 modes) or e4m3 bytes (NVFP4)
     const int32_t* slot_map;
     const int32_t* pad_rows;
     const int32_t* num_pad_rows;

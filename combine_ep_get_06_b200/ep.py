@@ -23,7 +23,7 @@ import torch
 from . import build as _build
 
 EP_OK, EP_ERR_INVALID_ARG, EP_ERR_DEVICE, EP_ERR_CUDA = 0, 1, 2, 3
-EP_X_BF16, EP_X_FP8, EP_X_BF16_TO_FP8 = 0, 1, 2
+EP_X_BF16, EP_X_FP8, EP_X_BF16_TO_FP8, EP_X_BF16_TO_NVFP4 = 0, 1, 2, 3
 EP_DEVERR_BAD_TOPK_IDX, EP_DEVERR_CAPACITY, EP_DEVERR_TIMEOUT = 1, 2, 4
 
 
@@ -252,10 +252,17 @@ def get_layout(topk_idx: torch.Tensor, num_experts: int, *, num_segments: int = 
 XType = Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]]
 
 
-def _dispatch_args(x: XType, handle: EPHandle, use_fp8: bool, recv_x, recv_scales, row_scales=True):
+def _bf16_mode(use_fp8: bool, use_nvfp4: bool) -> int:
+    if use_fp8 and use_nvfp4:
+        raise ValueError("use_fp8 and use_nvfp4 are exclusive")
+    return EP_X_BF16_TO_NVFP4 if use_nvfp4 else EP_X_BF16_TO_FP8 if use_fp8 else EP_X_BF16
+
+
+def _dispatch_args(x: XType, handle: EPHandle, bf16_mode: int, recv_x, recv_scales, row_scales=True):
     """Checks x and the receive buffers (allocating those not given);
-    returns (mode, x, x_scales, H, recv_x, recv_scales).  With row_scales
-    False the row-major recv_scales is neither checked nor allocated."""
+    returns (mode, x, x_scales, H, recv_x, recv_scales).  bf16_mode is the
+    mode a bf16 x takes.  With row_scales False the row-major recv_scales
+    is neither checked nor allocated."""
     dev = handle.device
     rows = handle.max_recv_rows
     x_scales = None
@@ -266,7 +273,7 @@ def _dispatch_args(x: XType, handle: EPHandle, use_fp8: bool, recv_x, recv_scale
         mode = EP_X_FP8
     else:
         _need(x, "x", (torch.bfloat16,), dev, 2)
-        mode = EP_X_BF16_TO_FP8 if use_fp8 else EP_X_BF16
+        mode = bf16_mode
     T, H = x.shape
     if T != handle.num_tokens:
         raise ValueError(f"x has {T} rows, handle has {handle.num_tokens} tokens")
@@ -276,6 +283,20 @@ def _dispatch_args(x: XType, handle: EPHandle, use_fp8: bool, recv_x, recv_scale
         if recv_x is None:
             recv_x = torch.empty(rows, H, dtype=torch.bfloat16, device=dev)
         _need(recv_x, "recv_x", (torch.bfloat16,), dev, 2)
+    elif mode == EP_X_BF16_TO_NVFP4:
+        if H % 32 != 0:
+            raise ValueError("NVFP4 dispatch needs hidden % 32 == 0")
+        if recv_x is None:
+            recv_x = torch.empty(rows, H // 2, dtype=torch.uint8, device=dev)
+        _need(recv_x, "recv_x", (torch.uint8,), dev, 2)
+        if tuple(recv_x.shape) != (rows, H // 2):
+            raise ValueError("recv_x must be [max_recv_rows, hidden/2] in the NVFP4 mode")
+        if recv_scales is None:
+            recv_scales = torch.empty(rows, H // 16, dtype=torch.uint8, device=dev)
+        _need(recv_scales, "recv_scales", (torch.uint8, torch.float8_e4m3fn), dev, 2)
+        if tuple(recv_scales.shape) != (rows, H // 16):
+            raise ValueError("recv_scales must be [max_recv_rows, hidden/16] in the NVFP4 mode")
+        return mode, x, x_scales, H, recv_x, recv_scales
     else:
         if recv_x is None:
             recv_x = torch.empty(rows, H, dtype=torch.float8_e4m3fn, device=dev)
@@ -291,14 +312,17 @@ def _dispatch_args(x: XType, handle: EPHandle, use_fp8: bool, recv_x, recv_scale
     return mode, x, x_scales, H, recv_x, recv_scales
 
 
-def dispatch_with_handle(x: XType, handle: EPHandle, *, use_fp8: bool = False,
+def dispatch_with_handle(x: XType, handle: EPHandle, *, use_fp8: bool = False, use_nvfp4: bool = False,
                          recv_x: Optional[torch.Tensor] = None,
                          recv_scales: Optional[torch.Tensor] = None):
     """Dispatch with an existing handle (decode with a cached handle; the
     backward of combine).  x bf16 [T,H] -> recv_x bf16 [max_recv_rows,H];
     x bf16 with use_fp8 -> (recv_x e4m3 [rows,H], recv_scales f32 [rows,H/128]);
+    x bf16 with use_nvfp4 -> (recv_x uint8 [rows,H/2] packed E2M1 pairs, the
+    even element in the low nibble, recv_scales uint8 e4m3 [rows,H/16]);
     x = (x_fp8 [T,H], scales [T,H/128]) -> the same tuple, copied."""
-    mode, x, x_scales, H, recv_x, recv_scales = _dispatch_args(x, handle, use_fp8, recv_x, recv_scales)
+    mode, x, x_scales, H, recv_x, recv_scales = _dispatch_args(x, handle, _bf16_mode(use_fp8, use_nvfp4),
+                                                               recv_x, recv_scales)
     _check(lib().ep_dispatch(handle.ref, mode, x.data_ptr(), _ptr(x_scales), H, recv_x.data_ptr(),
                              _ptr(recv_scales), _stream(handle.device)), "dispatch")
     return recv_x if mode == EP_X_BF16 else (recv_x, recv_scales)
@@ -307,7 +331,7 @@ def dispatch_with_handle(x: XType, handle: EPHandle, *, use_fp8: bool = False,
 def dispatch(x: XType, topk_idx: Optional[torch.Tensor] = None,
              topk_weights: Optional[torch.Tensor] = None, num_experts: Optional[int] = None, *,
              expert_alignment: int = 1, num_segments: int = 1, handle: Optional[EPHandle] = None,
-             use_fp8: bool = False, max_recv_rows: Optional[int] = None,
+             use_fp8: bool = False, use_nvfp4: bool = False, max_recv_rows: Optional[int] = None,
              recv_x: Optional[torch.Tensor] = None, recv_scales: Optional[torch.Tensor] = None,
              recv_topk_idx: Optional[torch.Tensor] = None,
              recv_topk_weights: Optional[torch.Tensor] = None):
@@ -318,7 +342,7 @@ def dispatch(x: XType, topk_idx: Optional[torch.Tensor] = None,
     if topk_idx is None:
         if handle is None:
             raise ValueError("dispatch needs topk_idx or a handle")
-        return dispatch_with_handle(x, handle, use_fp8=use_fp8, recv_x=recv_x,
+        return dispatch_with_handle(x, handle, use_fp8=use_fp8, use_nvfp4=use_nvfp4, recv_x=recv_x,
                                     recv_scales=recv_scales), None, None, handle
     if num_experts is None:
         raise ValueError("num_experts is required with topk_idx")
@@ -338,7 +362,8 @@ def dispatch(x: XType, topk_idx: Optional[torch.Tensor] = None,
     rw = torch.empty(R, dtype=torch.float32, device=dev) if recv_topk_weights is None else recv_topk_weights
     _need(ri, "recv_topk_idx", (torch.int32,), dev, 1)
     _need(rw, "recv_topk_weights", (torch.float32,), dev, 1)
-    mode, x, x_scales, H, recv_x, recv_scales = _dispatch_args(x, handle, use_fp8, recv_x, recv_scales)
+    mode, x, x_scales, H, recv_x, recv_scales = _dispatch_args(x, handle, _bf16_mode(use_fp8, use_nvfp4),
+                                                               recv_x, recv_scales)
     _check(lib().ep_layout_dispatch(handle.ref, topk_idx.data_ptr(), int(topk_idx.dtype == torch.int64),
                                     _ptr(topk_weights), ri.data_ptr(), rw.data_ptr(),
                                     handle.workspace_ptr, handle.workspace_bytes, mode, x.data_ptr(),
@@ -423,7 +448,7 @@ def dispatch_mn_scales(x: XType, handle: EPHandle, *, recv_x: Optional[torch.Ten
     _need(recv_scales_mn, "recv_scales_mn", (torch.float32,), dev, 2)
     if tuple(recv_scales_mn.shape) != (H // 128, scales_ld):
         raise ValueError("recv_scales_mn must be [hidden/128, scales_ld]")
-    mode, x, x_scales, H, recv_x, _ = _dispatch_args(x, handle, True, recv_x, None, row_scales=False)
+    mode, x, x_scales, H, recv_x, _ = _dispatch_args(x, handle, EP_X_BF16_TO_FP8, recv_x, None, row_scales=False)
     _check(lib().ep_dispatch_mn_scales(handle.ref, mode, x.data_ptr(), _ptr(x_scales), H, recv_x.data_ptr(),
                                        recv_scales_mn.data_ptr(), scales_ld, _stream(dev)), "dispatch_mn_scales")
     return recv_x, recv_scales_mn

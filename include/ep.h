@@ -74,9 +74,14 @@ typedef enum {
 typedef enum {
     EP_X_BF16 = 0,        /* x bf16 [T,H] -> recv_x bf16 [rows,H]; H % 8 == 0 */
     EP_X_FP8 = 1,         /* x e4m3 [T,H] + x_scales f32 [T,B] copied as they are; H % 128 == 0 */
-    EP_X_BF16_TO_FP8 = 2  /* x bf16 [T,H] quantised per 1x128 block: amax = max|x| floored at
+    EP_X_BF16_TO_FP8 = 2, /* x bf16 [T,H] quantised per 1x128 block: amax = max|x| floored at
                              1e-4, scale = amax/448, q = e4m3_rn_satfinite(x * (448/amax));
                              -> recv_x e4m3 [rows,H] + recv_scales f32 [rows,B]; H % 128 == 0 */
+    EP_X_BF16_TO_NVFP4 = 3 /* x bf16 [T,H] quantised to NVFP4 (the Hybrid-EP branch's NVFP4
+                             type): per 1x16 block amax = max|x| floored at 6*2^-9, scale =
+                             e4m3_rn_satfinite(amax/6), q = e2m1_rn_satfinite(x * (1/scale));
+                             -> recv_x [rows,H/2] bytes (two E2M1 codes each, the even element
+                             in the low nibble) + recv_scales [rows,H/16] e4m3 bytes; H % 32 == 0 */
 } ep_x_mode;
 
 /* Routing metadata of one layout (the pages' EPHandle).  A plain struct of
@@ -180,12 +185,14 @@ EP_API ep_status ep_get_layout_static(ep_handle* handle, const void* topk_idx, i
  * touched.
  *   x          [T,H] bf16 (EP_X_BF16, EP_X_BF16_TO_FP8) or e4m3 bytes (EP_X_FP8)
  *   x_scales   [T,B] f32 for EP_X_FP8, else ignored (may be NULL)
- *   recv_x     [max_recv_rows,H] bf16 (EP_X_BF16) or e4m3 bytes
- *   recv_scales [max_recv_rows,B] f32 for the FP8 modes, else ignored
+ *   recv_x     [max_recv_rows,H] bf16 (EP_X_BF16) or e4m3 bytes, or [max_recv_rows,H/2]
+ *              packed E2M1 (EP_X_BF16_TO_NVFP4)
+ *   recv_scales [max_recv_rows,B] f32 for the FP8 modes, [max_recv_rows,H/16] e4m3 bytes
+ *              for NVFP4, else ignored
  * The FP8 quantisation rounds to nearest-even with saturation at +-448. */
 EP_API ep_status ep_dispatch(const ep_handle* handle, ep_x_mode mode, const void* x,
                              const float* x_scales, int32_t hidden, void* recv_x,
-                             float* recv_scales, ep_stream_t stream);
+                             void* recv_scales, ep_stream_t stream);
 
 /* Layout and dispatch in one call: the dispatch(x, topk_idx, topk_weights,
  * num_experts, expert_alignment) call of the DeepEP V2 README ("Interfaces
@@ -199,12 +206,12 @@ EP_API ep_status ep_layout_dispatch(ep_handle* handle, const void* topk_idx, int
                                     float* recv_topk_weights, void* workspace,
                                     size_t workspace_bytes, ep_x_mode mode, const void* x,
                                     const float* x_scales, int32_t hidden, void* recv_x,
-                                    float* recv_scales, ep_stream_t stream);
+                                    void* recv_scales, ep_stream_t stream);
 
 /* Dispatch with the FP8 block scales laid out the way a grouped FP8 GEMM
  * reads them (DeepEP V2 README, "News": V2 adopts a new GEMM layout;
  * "Interfaces and examples": the per-expert counts feed the GEMM).  The same
- * as ep_dispatch in the two FP8 modes, except that the scale of block b of
+ * as ep_dispatch in the two FP8 modes (not NVFP4), except that the scale of block b of
  * receive row r goes to recv_scales_mn[b * scales_ld + r] (MN-major: one
  * column of rows per block).  scales_ld >= max_recv_rows and a multiple of
  * 4, so that every column starts 16-byte aligned for TMA; entries for rows
