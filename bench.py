@@ -67,6 +67,7 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-mgpu", action="store_true")
     return p.parse_args()
 
 
@@ -365,6 +366,8 @@ def run_ours(args, rank, world, dev):
                                "frac_of_peak": round(bwd_bytes / (bwd_ms * 1e-3) / 1e9 / peak, 4)}
     handle.check_error()
 
+    if not args.no_mgpu and H % 128 == 0:
+        res["mgpu_local"] = run_mgpu_local(args, dev, w, inp, nbytes)
     if not args.no_decode:
         res["decode"] = run_decode(args, dev)
     if not args.no_e2e:
@@ -372,6 +375,58 @@ def run_ours(args, rank, world, dev):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w, inp, y_np)
     return res
+
+
+def run_mgpu_local(args, dev, w, inp, nbytes, world=8):
+    """The multi-GPU dispatch / combine kernels with all `world` ranks'
+    blocks on this GPU: the step's batch split evenly over the ranks, so
+    the concatenated batch (and the algorithmic bytes) are the step's.
+    Times the dispatch phase (per-rank layouts, the counts exchange as
+    device copies, per-rank dispatch kernels) and the combine phase."""
+    import torch
+
+    import combine_ep_get_06_b200 as ep
+    from combine_ep_get_06_b200 import mgpu
+
+    def bf16(a, device):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+
+    T = inp["x"].shape[0]
+    if T % world:
+        return None
+    Tr = T // world
+    lr = mgpu.LocalRanks(world, Tr, w.k, w.E, w.H, expert_alignment=w.align, mode=ep.EP_X_BF16_TO_FP8,
+                         device=dev)
+    xs = [bf16(inp["x"][r * Tr:(r + 1) * Tr], dev) for r in range(world)]
+    idxs = [torch.from_numpy(inp["topk_idx"][r * Tr:(r + 1) * Tr].copy()).to(dev) for r in range(world)]
+    wts = [torch.from_numpy(inp["topk_weights"][r * Tr:(r + 1) * Tr].copy()).to(dev) for r in range(world)]
+    outs = [torch.empty(Tr, w.H, dtype=torch.bfloat16, device=dev) for _ in range(world)]
+    stream = torch.cuda.current_stream(dev)
+    for b in lr.blocks:
+        b.y.zero_()
+    for _ in range(3):
+        hs = lr.dispatch(xs, idxs, wts, use_fp8=True)
+        lr.combine(hs, wts, outs)
+    n = max(3, min(20, args.steps))
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    d_ms = c_ms = 0.0
+    for _ in range(n):
+        e[0].record(stream)
+        hs = lr.dispatch(xs, idxs, wts, use_fp8=True)
+        e[1].record(stream)
+        lr.combine(hs, wts, outs)
+        e[2].record(stream)
+        torch.cuda.synchronize(dev)
+        d_ms += e[0].elapsed_time(e[1])
+        c_ms += e[1].elapsed_time(e[2])
+    d_ms, c_ms = d_ms / n, c_ms / n
+    for r in lr.ranks:
+        r.check_error()
+    return {"config": f"{world} ranks x {Tr} tokens on one GPU, fp8 dispatch + bf16 combine",
+            "dispatch_phase_us": round(d_ms * 1e3, 2), "combine_us": round(c_ms * 1e3, 2),
+            "dispatch_phase_gbs": round(nbytes["dispatch"] / (d_ms * 1e-3) / 1e9, 1),
+            "combine_gbs": round(nbytes["combine"] / (c_ms * 1e-3) / 1e9, 1),
+            "launches_per_step": 2 * world + world + 1 + world + world}
 
 
 def run_decode(args, dev):

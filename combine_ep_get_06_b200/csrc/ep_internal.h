@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include "ep.h"
+#include "ep_multi.h"
 
 namespace ep {
 
@@ -89,6 +90,27 @@ struct CombineBackwardArgs {
 cudaError_t launch_combine_backward(const CombineBackwardArgs& a, cudaStream_t stream);
 
 // Number of SMs of the current device (cached per device).
+// Multi-GPU expert parallelism (include/ep_multi.h).
+constexpr int kMaxWorld = 128;
+
+struct MgpuArgs {
+    ep_mgpu_geometry g;       // by value
+    DispatchArgs src;         // x, x_scales, H (read by the dispatch item helpers)
+    int32_t T;                // this rank's tokens
+    const int32_t* slot_map;  // local handle (alignment 1): row among this rank's slots
+    const int32_t* offsets;   // local handle: first local row of each expert
+    const void* topk_idx;
+    int32_t idx_is_int64;
+    const float* topk_weights;
+    char* local_block;
+    char* const* peer_blocks; // device array [world]
+    void* out;                // combine output [T,H] bf16
+};
+
+size_t mgpu_dispatch_smem_bytes(const ep_mgpu_geometry& g);
+cudaError_t launch_mgpu_dispatch(const MgpuArgs& a, ep_x_mode mode, cudaStream_t stream);
+cudaError_t launch_mgpu_combine(const MgpuArgs& a, cudaStream_t stream);
+
 int device_sm_count();
 
 // Records a printf-style message for ep_last_error() and returns status.

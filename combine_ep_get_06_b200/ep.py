@@ -42,11 +42,24 @@ class _HandleC(ctypes.Structure):
                  "pad_rows", "num_pad_rows", "error_word")]
 
 
+class _GeomC(ctypes.Structure):
+    """ep_mgpu_geometry (include/ep_multi.h)."""
+    _fields_ = [(name, ctypes.c_int32) for name in
+                ("rank", "world", "max_tokens", "num_topk", "num_experts", "expert_alignment", "hidden",
+                 "x_mode", "experts_per_rank", "max_recv_rows", "row_bytes", "scale_bytes")] + \
+               [(name, ctypes.c_int64) for name in
+                ("off_recv_x", "off_recv_scales", "off_recv_src", "off_recv_topk_idx",
+                 "off_recv_topk_weights", "off_y", "off_all_counts", "off_dest", "off_raw_counts",
+                 "off_recv_counts", "off_recv_offsets", "off_num_pad_rows", "off_error_word",
+                 "block_bytes")]
+
+
 _LIB = None
 
 # name -> (restype, argtypes); mirrors include/ep.h
 _P, _I32, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
 _HP = ctypes.POINTER(_HandleC)
+_GP = ctypes.POINTER(_GeomC)
 SIGNATURES = {
     "ep_abi_version": (_I32, []),
     "ep_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -66,6 +79,17 @@ SIGNATURES = {
     "ep_read_recv_counts": (ctypes.c_int, [_HP, _P, _P]),
     "ep_read_total_rows": (ctypes.c_int, [_HP, ctypes.POINTER(_I32), _P]),
     "ep_check_error": (ctypes.c_int, [_HP, ctypes.POINTER(ctypes.c_uint32), _P]),
+    # include/ep_multi.h
+    "ep_mgpu_geometry_init": (ctypes.c_int, [_GP, _I32, _I32, _I32, _I32, _I32, _I32, _I32, ctypes.c_int]),
+    "ep_mgpu_block_alloc": (ctypes.c_int, [_SZ, ctypes.POINTER(_P)]),
+    "ep_mgpu_block_free": (ctypes.c_int, [_P]),
+    "ep_ipc_export": (ctypes.c_int, [_P, _P]),
+    "ep_ipc_import": (ctypes.c_int, [_P, ctypes.POINTER(_P)]),
+    "ep_ipc_close": (ctypes.c_int, [_P]),
+    "ep_mgpu_dispatch": (ctypes.c_int, [_GP, _HP, _P, _I32, _P, ctypes.c_int, _P, _P, _P, _P, _P]),
+    "ep_mgpu_combine": (ctypes.c_int, [_GP, _HP, _P, _P, _P, _P, _P]),
+    "ep_mgpu_read_total_rows": (ctypes.c_int, [_GP, _P, ctypes.POINTER(_I32), _P]),
+    "ep_mgpu_check_error": (ctypes.c_int, [_GP, _P, ctypes.POINTER(ctypes.c_uint32), _P]),
 }
 
 
