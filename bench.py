@@ -174,9 +174,10 @@ def nvsmi_device_id(dev) -> str | None:
 
 # ----------------------------------------------------------- ncu traffic
 
-def combine_traffic():
+def combine_traffic(workload: str, T: int):
     """Per-launch DRAM bytes of the combine kernel from the committed ncu
-    summary, if that summary was taken on the current combine source."""
+    summary, if that summary was taken on the current combine source and
+    on this workload."""
     src = os.path.join(ROOT, "combine_ep_get_06_b200", "csrc", "combine.cu")
     summ = os.path.join(ROOT, "profiles", "combine_kernel_v3.md")
     try:
@@ -186,6 +187,9 @@ def combine_traffic():
         return None
     m_sha = re.search(r"combine\.cu sha256\[:16\]:\s*`?([0-9a-f]{16})", text)
     m_tr = re.search(r"traffic per launch \(bytes\):\s*([0-9]+)", text)
+    m_wl = re.search(r"profiled workload:\s*(\w+) T=([0-9]+)", text)
+    if not (m_wl and m_wl.group(1) == workload and int(m_wl.group(2)) == T):
+        return None
     if m_sha and m_tr and m_sha.group(1) == sha:
         return int(m_tr.group(1))
     return None
@@ -303,7 +307,7 @@ def run_ours(args, rank, world, dev):
     achieved = nbytes["combine"] / (com_ms * 1e-3) / 1e9
     res["roofline"] = {"bound": "hbm", "kernel": "combine_kernel", "achieved": round(achieved, 1),
                        "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                       "frac": round(achieved / peak, 4), "traffic": combine_traffic(),
+                       "frac": round(achieved / peak, 4), "traffic": combine_traffic(w.name, T),
                        "algorithmic_bytes": nbytes["combine"]}
 
     # FP8 dispatch with GEMM-ready (MN-major) scales, same workload

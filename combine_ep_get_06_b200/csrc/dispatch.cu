@@ -35,16 +35,25 @@ __host__ __device__ inline size_t smem_bytes(const Geometry& g) {
 
 // Stores the scale of block b of receive row `row` (f32 row- or MN-major,
 // or an e4m3 byte for NVFP4), taken from the row's scale buffer sb.
+// MN-major scales are stored with an L2 evict-last policy: each token's
+// scales land in B different columns, 4 bytes per 32-byte sector, and the
+// whole array fits in L2, so its sectors fill up there before write-back
+// (measured: 158 -> 134 us at the V3 shape).  A hint on the row copies
+// measured slower and is not used.
 template <int kMode>
-__device__ __forceinline__ void store_scale(const DispatchArgs& a, int row, int b, const float* sb, bool zero) {
+__device__ __forceinline__ void store_scale(const DispatchArgs& a, int row, int b, const float* sb, bool zero,
+                                            uint64_t keep) {
     if (kMode == EP_X_BF16_TO_NVFP4) {
         reinterpret_cast<unsigned char*>(a.recv_scales)[(size_t)row * (a.H / 16) + b] =
             zero ? 0 : reinterpret_cast<const unsigned char*>(sb)[b];
+    } else if (a.scales_ld > 0) {
+        st_f32_hint(reinterpret_cast<float*>(a.recv_scales) + (size_t)b * a.scales_ld + row, zero ? 0.0f : sb[b],
+                    keep);
     } else {
-        const size_t at = a.scales_ld > 0 ? (size_t)b * a.scales_ld + row : (size_t)row * (a.H / 128) + b;
-        reinterpret_cast<float*>(a.recv_scales)[at] = zero ? 0.0f : sb[b];
+        reinterpret_cast<float*>(a.recv_scales)[(size_t)row * (a.H / 128) + b] = zero ? 0.0f : sb[b];
     }
 }
+
 
 template <int kMode>
 __device__ __forceinline__ void prefetch(const DispatchArgs& a, int t, int ipr, Item (&p)[kPre]) {
@@ -75,6 +84,7 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchArgs a) {
     for (int i = tid; i < (geo.row_bytes + geo.scale_pad) / 16; i += kThreads)
         reinterpret_cast<uint4*>(zeros)[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
+    const uint64_t keep = a.scales_ld > 0 ? l2_evict_last_policy() : 0;
 
     // Right after the layout x is already complete (every layout kernel waits
     // for the grid before it before letting this one launch), so the first
@@ -101,7 +111,7 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchArgs a) {
                         bulk_s2g(rscl + (size_t)row * geo.scale_bytes, zeros + geo.row_bytes, geo.scale_bytes);
                     bulk_commit();
                     if (kFp8Out && !a.bulk_scales)
-                        for (int b = 0; b < B; ++b) store_scale<kMode>(a, row, b, nullptr, true);
+                        for (int b = 0; b < B; ++b) store_scale<kMode>(a, row, b, nullptr, true, keep);
                 }
             }
             continue;
@@ -149,7 +159,7 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchArgs a) {
             // MN-major scales, or rows not a multiple of 16 bytes: plain stores.
             for (int i = tid; i < k * B; i += kThreads) {
                 const int row = rows[i / B];
-                if (row >= 0 && row < a.max_rows) store_scale<kMode>(a, row, i % B, sb, false);
+                if (row >= 0 && row < a.max_rows) store_scale<kMode>(a, row, i % B, sb, false, keep);
             }
         }
     }
