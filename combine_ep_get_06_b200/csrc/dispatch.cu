@@ -26,11 +26,12 @@ using namespace dispatch_dev;
 
 constexpr int kThreads = 256;
 constexpr int kPre = 2;  // 32-item slices per warp whose loads are prefetched
+constexpr int kBuf = 2;  // row buffers: a buffer is refilled once the copies from kBuf rows ago have read it
 
-// smem: [2][row_bytes] row buffers | [2][scale_pad] scale buffers |
-//       [row_bytes] zeros | [scale_pad] zeros | [2][kMaxTopk] int rows
+// smem: [kBuf][row_bytes] row buffers | [kBuf][scale_pad] scale buffers |
+//       [row_bytes] zeros | [scale_pad] zeros | [kBuf][kMaxTopk] int rows
 __host__ __device__ inline size_t smem_bytes(const Geometry& g) {
-    return (size_t)3 * g.row_bytes + (size_t)3 * g.scale_pad + 2 * kMaxTopk * sizeof(int);
+    return (size_t)(kBuf + 1) * g.row_bytes + (size_t)(kBuf + 1) * g.scale_pad + kBuf * kMaxTopk * sizeof(int);
 }
 
 // Stores the scale of block b of receive row `row` (f32 row- or MN-major,
@@ -70,10 +71,10 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchArgs a) {
     constexpr bool kFp8Out = kMode != EP_X_BF16;
     extern __shared__ __align__(128) unsigned char smem[];
     const Geometry geo = geometry(kMode, a.H);
-    unsigned char* rowbuf = smem;                                  // [2][row_bytes]
-    unsigned char* sclbuf = smem + 2 * geo.row_bytes;              // [2][scale_pad]
-    unsigned char* zeros = sclbuf + 2 * geo.scale_pad;             // [row_bytes + scale_pad]
-    int* rows_s = (int*)(zeros + geo.row_bytes + geo.scale_pad);   // [2][kMaxTopk]
+    unsigned char* rowbuf = smem;                                  // [kBuf][row_bytes]
+    unsigned char* sclbuf = smem + kBuf * geo.row_bytes;           // [kBuf][scale_pad]
+    unsigned char* zeros = sclbuf + kBuf * geo.scale_pad;          // [row_bytes + scale_pad]
+    int* rows_s = (int*)(zeros + geo.row_bytes + geo.scale_pad);   // [kBuf][kMaxTopk]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int T = a.T, k = a.k;
@@ -118,14 +119,15 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchArgs a) {
         }
 
         const int t = r;
-        const int buf = it & 1;
+        const int buf = it % kBuf;
         ++it;
         unsigned char* rb = rowbuf + buf * geo.row_bytes;
         float* sb = reinterpret_cast<float*>(sclbuf + buf * geo.scale_pad);
         int* rows = rows_s + buf * kMaxTopk;
 
-        // The copies issued two rows ago from this buffer must have read it.
-        if (warp == 0) bulk_wait_read<1>();
+        // The copies issued kBuf rows ago from this buffer must have read it
+        // (each lane below k commits one bulk group per token row).
+        if (warp == 0) bulk_wait_read<kBuf - 1>();
         __syncthreads();
 
         if (tid < k) rows[tid] = ld_cg(a.slot_map + (size_t)t * k + tid);

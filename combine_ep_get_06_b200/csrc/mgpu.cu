@@ -282,8 +282,11 @@ __global__ void __launch_bounds__(kThreads) mgpu_dispatch_kernel(MgpuArgs a) {
                          tid, kThreads);
         }
     }
-    // the stores to peers' memory are complete before the grid is
-    __threadfence_system();
+    // The CTA's stores to peers' memory are ordered before the grid's end:
+    // the barrier makes them precede thread 0's system-scope fence, which is
+    // cumulative.  (A fence in every thread measured as the top stall.)
+    __syncthreads();
+    if (tid == 0) __threadfence_system();
 }
 
 template <int G>

@@ -215,12 +215,14 @@ class RankEP:
 
 class LocalRanks:
     """W ranks with all blocks on one GPU.  The peer table holds plain
-    device addresses, the all-gather is a device copy, and the ranks'
-    launches run one after another on the current stream.  No kernel waits
-    on another."""
+    device addresses and the all-gather is a device copy.  The ranks'
+    launches run one after another on the current stream, or, with
+    ``concurrent``, each rank's on a stream of its own, joined by events
+    around the exchange and at the end.  No kernel waits on another."""
 
     def __init__(self, world: int, max_tokens: int, num_topk: int, num_experts: int, hidden: int, *,
-                 expert_alignment: int = 1, mode: int = EP_X_BF16_TO_FP8, device=None):
+                 expert_alignment: int = 1, mode: int = EP_X_BF16_TO_FP8, device=None,
+                 concurrent: bool = False):
         device = torch.device("cuda") if device is None else torch.device(device)
         if device.index is None:
             device = torch.device("cuda", torch.cuda.current_device())
@@ -232,6 +234,22 @@ class LocalRanks:
                        for g in self.geoms]
         self.peers = torch.tensor([b.ptr for b in self.blocks], dtype=torch.int64, device=device)
         self.ranks = [RankEP(g, b, self.peers) for g, b in zip(self.geoms, self.blocks)]
+        self.streams = [torch.cuda.Stream(device) for _ in range(world)] if concurrent else None
+
+    def _per_rank(self, fn):
+        """fn(r) for every rank: in order on the current stream, or each on
+        its own stream after the current stream's work, joined back."""
+        if self.streams is None:
+            return [fn(r) for r in range(self.world)]
+        main = torch.cuda.current_stream(self.device)
+        out = []
+        for r, s in enumerate(self.streams):
+            s.wait_stream(main)
+            with torch.cuda.stream(s):
+                out.append(fn(r))
+        for s in self.streams:
+            main.wait_stream(s)
+        return out
 
     def exchange_counts(self, handles: Sequence[EPHandle]):
         """The all-gather of step 2, as device copies."""
@@ -240,17 +258,17 @@ class LocalRanks:
             b.all_counts.copy_(stacked)
 
     def dispatch(self, xs, topk_idxs, topk_weights=None, *, use_fp8=False, use_nvfp4=False) -> List[EPHandle]:
-        handles = [r.layout(i) for r, i in zip(self.ranks, topk_idxs)]
+        handles = self._per_rank(lambda r: self.ranks[r].layout(topk_idxs[r]))
         self.exchange_counts(handles)
         ws = topk_weights if topk_weights is not None else [None] * self.world
-        for r, h, x, i, w in zip(self.ranks, handles, xs, topk_idxs, ws):
-            r.dispatch(h, x, i, w, use_fp8=use_fp8, use_nvfp4=use_nvfp4)
+        self._per_rank(lambda r: self.ranks[r].dispatch(handles[r], xs[r], topk_idxs[r], ws[r], use_fp8=use_fp8,
+                                                        use_nvfp4=use_nvfp4))
         return handles
 
     def combine(self, handles, topk_weights=None, outs=None):
         ws = topk_weights if topk_weights is not None else [None] * self.world
         os_ = outs if outs is not None else [None] * self.world
-        return [r.combine(h, w, o) for r, h, w, o in zip(self.ranks, handles, ws, os_)]
+        return self._per_rank(lambda r: self.ranks[r].combine(handles[r], ws[r], os_[r]))
 
 
 class _TorchComm:

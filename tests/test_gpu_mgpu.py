@@ -205,3 +205,36 @@ def test_capacity_error_when_counts_are_not_from_this_step():
     for b in lr.blocks:
         assert bool((b.mem[g.off_recv_scales: g.off_recv_src] == SENTINEL).all())
         assert bool((b.y.view(torch.uint8) == SENTINEL).all())
+
+
+def test_concurrent_ranks_give_the_same_bytes():
+    # each rank's launches on a stream of its own (joined by events around
+    # the exchange): identical blocks and outputs to the sequential form
+    w = W.WORKLOADS["mid"]
+    world, Ts = 4, [800, 640, 1024, 512]
+    inps = [W.make_inputs(w, seed=60 + r, T=Ts[r]) for r in range(world)]
+    xs = [to_dev_bf16(i["x"]) for i in inps]
+    idxs = [torch.from_numpy(i["topk_idx"]).cuda() for i in inps]
+    wts = [torch.from_numpy(i["topk_weights"]).cuda() for i in inps]
+    ys = None
+    res = []
+    for concurrent in (False, True):
+        lr = mgpu.LocalRanks(world, 1024, w.k, w.E, w.H, expert_alignment=w.align, concurrent=concurrent)
+        for b in lr.blocks:
+            b.mem.fill_(SENTINEL)
+            b.error_word.zero_()
+        hs = lr.dispatch(xs, idxs, wts, use_fp8=True)
+        if ys is None:
+            ys = [torch.randn(b.y.shape, device="cuda").to(torch.bfloat16) for b in lr.blocks]
+        for b, y in zip(lr.blocks, ys):
+            b.y.copy_(y)
+        outs = lr.combine(hs, wts)
+        torch.cuda.synchronize()
+        g = lr.geoms[0]
+        res.append(([b.mem[: g.off_y].clone() for b in lr.blocks],
+                    [b.mem[g.off_all_counts: g.block_bytes].clone() for b in lr.blocks], outs))
+    for a, b in zip(res[0][0] + res[0][1], res[1][0] + res[1][1]):
+        assert torch.equal(a, b)
+    for a, b in zip(res[0][2], res[1][2]):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
