@@ -64,7 +64,7 @@ def parse_args():
                    help="override the workload's token count (same shapes otherwise; for profiling)")
     p.add_argument("--decode-pairs", type=int, default=256)
     p.add_argument("--decode-replays", type=int, default=20)
-    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--e2e-steps", type=int, default=8)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
@@ -545,7 +545,11 @@ def run_e2e(args, dev, w, inp, y_np, nbytes):
     """Same metric through the public API with HOST inputs: every step
     copies x, topk_idx, topk_weights and y from pinned host memory, runs
     layout -> dispatch -> combine, and copies recv_x, recv_scales and the
-    combined output back to pinned host memory."""
+    combined output back to pinned host memory.  Steps are pipelined the
+    way a host-fed job runs them: two sets of device buffers, and the
+    copies in (one stream), kernels (another) and copies out (a third)
+    overlap across consecutive steps.  A set is refilled only after its
+    previous step's kernels and copies out have finished (events)."""
     import torch
 
     import combine_ep_get_06_b200 as ep
@@ -556,46 +560,79 @@ def run_e2e(args, dev, w, inp, y_np, nbytes):
     hi = torch.from_numpy(inp["topk_idx"]).pin_memory()
     hw = torch.from_numpy(inp["topk_weights"]).pin_memory()
     hy = torch.from_numpy(np.ascontiguousarray(y_np).view(np.int16)).view(torch.bfloat16).pin_memory()
-    handle = ep.EPHandle(T, k, w.E, w.S, w.align, device=dev)
-    rows = handle.max_recv_rows
-    dx = torch.empty_like(hx, device=dev)
-    di = torch.empty_like(hi, device=dev)
-    dw = torch.empty_like(hw, device=dev)
-    dy = torch.empty_like(hy, device=dev)
-    rq = torch.empty(rows, H, dtype=torch.float8_e4m3fn if fp8 else torch.bfloat16, device=dev)
-    rs = torch.empty(rows, H // 128, dtype=torch.float32, device=dev) if fp8 else None
-    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
-    h_rq = torch.empty(rq.shape, dtype=rq.dtype).pin_memory()
-    h_rs = torch.empty(rs.shape, dtype=rs.dtype).pin_memory() if fp8 else None
-    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    rows = ep.max_recv_rows(T, k, w.E, w.align)
+    qdt = torch.float8_e4m3fn if fp8 else torch.bfloat16
+
+    def device_set():
+        return {"handle": ep.EPHandle(T, k, w.E, w.S, w.align, device=dev),
+                "x": torch.empty_like(hx, device=dev), "i": torch.empty_like(hi, device=dev),
+                "w": torch.empty_like(hw, device=dev), "y": torch.empty_like(hy, device=dev),
+                "rq": torch.empty(rows, H, dtype=qdt, device=dev),
+                "rs": torch.empty(rows, H // 128, dtype=torch.float32, device=dev) if fp8 else None,
+                "out": torch.empty(T, H, dtype=torch.bfloat16, device=dev),
+                "in_done": torch.cuda.Event(), "disp_done": torch.cuda.Event(),
+                "comp_done": torch.cuda.Event(), "out_done": torch.cuda.Event()}
+
+    sets = [device_set(), device_set()]
+    h_rq = torch.empty(rows, H, dtype=qdt).pin_memory()
+    h_rs = torch.empty(rows, H // 128, dtype=torch.float32).pin_memory() if fp8 else None
+    h_out = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
     h2d = hx.numel() * 2 + hi.numel() * 8 + hw.numel() * 4 + hy.numel() * 2
     d2h = h_rq.numel() * h_rq.element_size() + (h_rs.numel() * 4 if fp8 else 0) + h_out.numel() * 2
+    s_in, s_k, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def step():
-        dx.copy_(hx, non_blocking=True)
-        di.copy_(hi, non_blocking=True)
-        dw.copy_(hw, non_blocking=True)
-        ep.get_layout(di, w.E, num_segments=w.S, expert_alignment=w.align, topk_weights=dw, handle=handle)
-        ep.dispatch_with_handle(dx, handle, use_fp8=fp8, recv_x=rq, recv_scales=rs)
-        h_rq.copy_(rq, non_blocking=True)
-        if fp8:
-            h_rs.copy_(rs, non_blocking=True)
-        dy.copy_(hy, non_blocking=True)
-        ep.combine(dy, handle, dw, out=out)
-        h_out.copy_(out, non_blocking=True)
+    def step(i):
+        d = sets[i % 2]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(d["comp_done"])       # the set's last kernels have read its inputs
+            d["x"].copy_(hx, non_blocking=True)
+            d["i"].copy_(hi, non_blocking=True)
+            d["w"].copy_(hw, non_blocking=True)
+            d["y"].copy_(hy, non_blocking=True)
+            d["in_done"].record(s_in)
+        with torch.cuda.stream(s_k):
+            s_k.wait_event(d["in_done"])
+            if i >= 2:
+                s_k.wait_event(d["out_done"])         # its outputs have been copied out
+            ep.get_layout(d["i"], w.E, num_segments=w.S, expert_alignment=w.align, topk_weights=d["w"],
+                          handle=d["handle"])
+            ep.dispatch_with_handle(d["x"], d["handle"], use_fp8=fp8, recv_x=d["rq"], recv_scales=d["rs"])
+            d["disp_done"].record(s_k)
+            ep.combine(d["y"], d["handle"], d["w"], out=d["out"])
+            d["comp_done"].record(s_k)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(d["disp_done"])
+            h_rq.copy_(d["rq"], non_blocking=True)
+            if fp8:
+                h_rs.copy_(d["rs"], non_blocking=True)
+            s_out.wait_event(d["comp_done"])
+            h_out.copy_(d["out"], non_blocking=True)
+            d["out_done"].record(s_out)
 
-    step()
+    main = torch.cuda.current_stream(dev)
+    for s_ in (s_in, s_k, s_out):
+        s_.wait_stream(main)
+    for i in range(2):
+        step(i)
+    for s_ in (s_in, s_k, s_out):
+        main.wait_stream(s_)
     torch.cuda.synchronize(dev)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(args.e2e_steps):
-        step()
-    b.record()
+    a.record(main)
+    for s_ in (s_in, s_k, s_out):
+        s_.wait_stream(main)
+    for i in range(args.e2e_steps):
+        step(i)
+    for s_ in (s_in, s_k, s_out):
+        main.wait_stream(s_)
+    b.record(main)
     torch.cuda.synchronize(dev)
     ms = a.elapsed_time(b) / args.e2e_steps
     total = sum(nbytes.values())
     return {"value": round(total / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(ms, 3),
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+            "pipelined": "copies in / kernels / copies out on three streams, two buffer sets"}
 
 
 # ------------------------------------------------------ CPU oracle timing
