@@ -6,7 +6,7 @@ on every rank; the dispatch kernel stores rows into the owners' blocks and
 the combine kernel loads expert outputs from them, through a device table
 of the W blocks' addresses.
 
-Three layers:
+Layers:
   * ``Geometry`` / ``RankBlock``: one rank's block and tensor views of its
     sections (receive rows, scales, metadata, y, totals).
   * ``RankEP``: the per-rank calls -- layout, dispatch, combine -- given a
@@ -14,7 +14,7 @@ Three layers:
   * ``ExpertParallelGroup``: one process per GPU over torch.distributed.
     It exchanges the blocks by CUDA IPC, all-gathers the per-expert counts
     before each dispatch, and runs the barriers the ordering needs.
-    ``LocalRanks``: all W ranks' blocks on one GPU, with the all-gather
+  * ``LocalRanks``: all W ranks' blocks on one GPU, with the all-gather
     done as device copies.  This is the form the one-GPU tests and the
     benchmark run.
 """
@@ -26,7 +26,7 @@ from typing import List, Optional, Sequence
 
 import torch
 
-from .ep import (EP_X_BF16, EP_X_BF16_TO_FP8, EP_X_BF16_TO_NVFP4, EP_X_FP8, EPError, EPHandle, _GeomC,
+from .ep import (EP_X_BF16, EP_X_BF16_TO_FP8, EP_X_BF16_TO_NVFP4, EP_X_FP8, EPHandle, _GeomC,
                  _check, _need, _ptr, _stream, lib)
 
 IPC_HANDLE_BYTES = 64

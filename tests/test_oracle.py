@@ -10,7 +10,6 @@ unweighted combine are adjoint, FP8 round trip).
 """
 
 import json
-import math
 import os
 from fractions import Fraction
 
