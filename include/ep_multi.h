@@ -85,7 +85,7 @@ typedef struct ep_mgpu_geometry {
 } ep_mgpu_geometry;
 
 /* Fills *g.  Limits: 0 <= rank < world, world >= 1 and divides E,
- * 1 <= E/world <= 1024, E <= 1024 * world, max_tokens >= 0, 1 <= k <= 32,
+ * 1 <= E <= 1024, world <= 128, max_tokens >= 0, 1 <= k <= 32,
  * a >= 1, hidden as ep_dispatch requires for x_mode, and W*max_tokens*k
  * + (E/W)*(a-1) < 2^31.  Host only. */
 EP_API ep_status ep_mgpu_geometry_init(ep_mgpu_geometry* g, int32_t rank, int32_t world,
@@ -99,8 +99,8 @@ EP_API ep_status ep_mgpu_block_alloc(size_t bytes, void** block);
 EP_API ep_status ep_mgpu_block_free(void* block);
 
 /* CUDA IPC of a rank block (not multicast): ep_ipc_export writes
- * EP_IPC_HANDLE_BYTES bytes that another process on another GPU of the
- * same node passes to ep_ipc_import, which maps the block into that
+ * EP_IPC_HANDLE_BYTES bytes that another process, on this GPU or another
+ * one of the node, passes to ep_ipc_import, which maps the block into that
  * process (peer access enabled lazily) and returns its address there.
  * ep_ipc_close unmaps an imported block.  A block cannot be imported by
  * the process that allocated it: use its own address there. */
@@ -122,7 +122,9 @@ EP_API ep_status ep_ipc_close(void* block);
  * Writes this rank's dest and, from all_counts, its own receive totals
  * (raw_counts, recv_counts, recv_offsets, num_pad_rows) and its own padding rows.
  * A computed row >= max_recv_rows (all_counts not from this step's all-gather)
- * sets EP_DEVERR_CAPACITY in the block's error word and is skipped. */
+ * sets EP_DEVERR_CAPACITY in the block's error word and is skipped; a
+ * topk_idx value outside [0, E) on a slot the layout kept (a topk_idx that
+ * is not the layout's) sets EP_DEVERR_BAD_TOPK_IDX and drops the slot. */
 EP_API ep_status ep_mgpu_dispatch(const ep_mgpu_geometry* g, const ep_handle* local,
                                   const void* topk_idx, int32_t idx_is_int64,
                                   const float* topk_weights, ep_x_mode mode, const void* x,
