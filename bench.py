@@ -97,6 +97,22 @@ def step_bytes(w: W.Workload, T: int, V: int, P: int, R: int) -> dict:
     return {"layout": layout, "dispatch": dispatch, "combine": combine}
 
 
+def step_config(w: W.Workload, T: int, world: int) -> dict:
+    """The `config` object of the JSON line (both arms)."""
+    return {"workload": f"{w.name}: T={T} hidden={w.H} experts={w.E} segments={w.S} "
+                        f"topk={w.k} alignment={w.align} x={w.x_mode}",
+            "T": T, "hidden": w.H, "experts": w.E, "segments": w.S, "topk": w.k, "alignment": w.align,
+            "dispatch": "bf16 -> e4m3 1x128" if w.x_mode == "fp8_quant" else "bf16",
+            "combine": "bf16, weighted, fp32 accumulation", "parallelism": f"replicas{world}",
+            "l2": "no flush: each step touches ~1.8 GB, > 126 MB L2"}
+
+
+def layout_launches(T: int, k: int) -> int:
+    """Kernels per layout: one CTA does it all when the slots fit one chunk
+    of 1024 (T <= 1024 // k), else a count and an assign kernel."""
+    return 1 if T <= 1024 // k else 2
+
+
 def max_over_ranks(x: float, world: int, device) -> float:
     """The largest x over all ranks (the slowest rank's time); x itself at N=1."""
     if world == 1:
@@ -288,13 +304,8 @@ def run_ours(args, rank, world, dev):
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": f"{w.name}: T={T} hidden={H} experts={w.E} segments={w.S} "
-                               f"topk={k} alignment={w.align} x={w.x_mode}",
-                   "T": T, "hidden": H, "experts": w.E, "segments": w.S, "topk": k,
-                   "alignment": w.align, "dispatch": "bf16 -> e4m3 1x128" if fp8 else "bf16",
-                   "combine": "bf16, weighted, fp32 accumulation", "parallelism": f"replicas{world}",
-                   "l2": "no flush: each step touches ~1.8 GB, > 126 MB L2"},
-        "gpu_launches": K * (4 if handle.c.num_tokens * k > 2048 else 3),
+        "config": step_config(w, T, world),
+        "gpu_launches": K * (layout_launches(T, k) + 2),
         "layout_us": round(lay_ms * 1e3, 2),
         "dispatch": {"us": round(dis_ms * 1e3, 2), "bytes": nbytes["dispatch"],
                      "gbs": round(nbytes["dispatch"] / (dis_ms * 1e-3) / 1e9, 1),
@@ -677,6 +688,9 @@ def run_reference(args):
     token sample of the same workload per step (sized so that the whole
     run stays within about two minutes)."""
     w = W.WORKLOADS[args.workload]
+    if args.tokens is not None:
+        w = dataclasses.replace(w, T=args.tokens)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     probe_T = 64
     inp = W.make_inputs(w, seed=0, T=probe_T)
     y_np = W.make_y(w, seed=0, rows=W.y_rows(W.Workload(**{**w.__dict__, "T": probe_T})))
@@ -701,8 +715,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_t / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": f"{w.name}: T={w.T} hidden={w.H} experts={w.E} segments={w.S} "
-                               f"topk={w.k} alignment={w.align} x={w.x_mode}"},
+        "config": step_config(w, w.T, world),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
