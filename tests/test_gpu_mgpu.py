@@ -238,3 +238,12 @@ def test_concurrent_ranks_give_the_same_bytes():
     for a, b in zip(res[0][2], res[1][2]):
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
+
+
+@pytest.mark.parametrize("world,E,k", [(16, 64, 12), (64, 64, 32), (3, 48, 20), (2, 64, 9)])
+def test_many_ranks_large_topk(world, E, k):
+    # k > 8 takes the combine's 2-4 groups of 8 slots; E/W down to one expert per rank
+    w = dataclasses.replace(W.WORKLOADS["tiny"], name=f"w{world}_e{E}_k{k}", E=E, S=world, k=k, align=4)
+    # blocks hold world * max_tokens * k rows each: few tokens per rank when many ranks
+    Ts = [8 + r % 5 for r in range(world)] if world >= 16 else [40 + 3 * r for r in range(world)]
+    run_case(w, world, Ts, "bf16", seed=world + k)
