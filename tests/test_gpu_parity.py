@@ -83,6 +83,8 @@ EDGE = [
     (5000, 4, 1024, 1024, 1, 64, "bf16", 0.0),       # many chunks, S = E
     (3000, 8, 8, 2, 512, 512, "fp8_quant", 0.0),     # alignment larger than most counts
     (2049, 1, 3, 1, 5, 1024, "fp8_quant", 1.0),      # every slot dropped
+    (131072, 8, 256, 8, 128, 128, "fp8_quant", 0.01),  # 1M slots: 1024 layout chunks
+    (65536, 8, 1024, 32, 16, 64, "bf16", 0.0),        # 512 chunks x 1024 experts
 ]
 
 
