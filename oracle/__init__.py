@@ -62,6 +62,8 @@ def lib():
         L.oracle_dispatch.restype = None
         L.oracle_combine.argtypes = [i32, i32, i32, P, P, P, P, P, P]
         L.oracle_combine.restype = None
+        L.oracle_combine_fp8.argtypes = [i32, i32, i32, P, P, P, P, P]
+        L.oracle_combine_fp8.restype = None
         L.oracle_combine_backward.argtypes = [i32, i32, i32, i32, P, P, P, P, P, P, P]
         L.oracle_combine_backward.restype = None
         _lib = L
@@ -210,6 +212,19 @@ def combine(slot_map: np.ndarray, T: int, k: int, y: np.ndarray, weights=None,
     ow = np.empty((T, k), np.float32) if want_out_weights else None
     lib().oracle_combine(T, k, H, _p(sm), _p(y), _p(w), _p(rw), _p(ow), _p(out))
     return out, ow
+
+
+def combine_fp8(slot_map: np.ndarray, T: int, k: int, yq: np.ndarray, ys: np.ndarray, weights=None):
+    """FP8 expert outputs (e4m3 codes [rows, H], f32 scales [rows, H/128])
+    -> out bf16 bits [T, H]."""
+    q = _c(yq, np.uint8)
+    H = q.shape[1]
+    s = _c(ys, np.float32)
+    sm = _c(slot_map, np.int32)
+    w = None if weights is None else _c(weights, np.float32)
+    out = np.empty((T, H), np.uint16)
+    lib().oracle_combine_fp8(T, k, H, _p(sm), _p(q), _p(s), _p(w), _p(out))
+    return out
 
 
 def combine_backward(lay: dict, grad_out: np.ndarray, y: np.ndarray, weights: np.ndarray):

@@ -54,6 +54,11 @@
  *     inv = 1 / scale (one IEEE division), q = e2m1(x * inv) rounded to
  *     nearest-even and saturating at +-6; two codes per byte, the even
  *     element in the low nibble;
+ *   - FP8 combine (the README's introduction says the kernels support low
+ *     precision, FP8 included; nothing fixes the combine's arithmetic):
+ *     expert outputs as e4m3 codes with one f32 scale per 1x128 block, the
+ *     same layout as the FP8 dispatch's output; v = e4m3_decode(q) * scale
+ *     (one binary32 multiply), then the combine sum above;
  *   - combine backward: grad_y[row] = bf16(w * g) with the product taken in
  *     binary32 (one multiply, one bf16 rounding); padding rows of grad_y are
  *     zero; grad_w is the exact dot product, accumulated here in binary64
@@ -386,6 +391,32 @@ EXPORT void oracle_combine(int32_t T, int32_t k, int32_t H, const int32_t* slot_
             for (int32_t j = 0; j < k; ++j)
                 out_weights[(int64_t)t * k + j] =
                     (sm[j] >= 0 && recv_weights_in) ? recv_weights_in[sm[j]] : 0.0f;
+    }
+}
+
+/* Combine of FP8 expert outputs (the low-precision combine: DeepEP V2
+ * README, introduction -- the kernels support low precision, FP8 included).
+ * Row r of y holds e4m3 codes yq[r, :] and one f32 scale per 1x128 block,
+ * ys[r, b].  Each value is decoded and multiplied by its block's scale in
+ * binary32 (one rounding), then accumulated as in oracle_combine:
+ *   v = e4m3_decode(yq[r,h]) * ys[r, h/128]
+ *   out[t,h] = bf16( acc ),  acc = fmaf(w[t,j], v, acc) from +0 over valid j ascending.
+ * With weights NULL every w is 1. */
+EXPORT void oracle_combine_fp8(int32_t T, int32_t k, int32_t H, const int32_t* slot_map, const uint8_t* yq,
+                               const float* ys, const float* weights, uint16_t* out) {
+    const int32_t B = H / 128;
+    for (int32_t t = 0; t < T; ++t) {
+        for (int32_t h = 0; h < H; ++h) {
+            float sum = 0.0f;
+            for (int32_t j = 0; j < k; ++j) {
+                const int32_t r = slot_map[(int64_t)t * k + j];
+                if (r < 0) continue;
+                const float wj = weights ? weights[(int64_t)t * k + j] : 1.0f;
+                const float v = oracle_e4m3_decode(yq[(size_t)r * H + h]) * ys[(size_t)r * B + h / 128];
+                sum = fmaf(wj, v, sum);
+            }
+            out[(size_t)t * H + h] = oracle_f32_to_bf16(sum);
+        }
     }
 }
 

@@ -427,6 +427,84 @@ def test_combine_equals_exact_rational_fma_chain():
         assert np.array_equal(out, bf16_bits_of(exp))
 
 
+def _e4m3_codes(rng, shape):
+    """Random e4m3 codes, both signs, no NaN (0x7F / 0xFF)."""
+    c = rng.integers(0, 0x7F, size=shape).astype(np.uint8)
+    return c | (rng.integers(0, 2, size=shape).astype(np.uint8) << 7)
+
+
+def test_combine_fp8_with_power_of_two_scales_is_the_bf16_combine_of_the_decoded_values():
+    # With a power-of-two scale, decode(q) * scale is exact and fits bf16
+    # (3 mantissa bits in 7), so the FP8 combine must equal the bf16 combine
+    # of those values.  The decode here is torch's, not the oracle's, and
+    # every 128-column block gets its own scale.
+    rng = np.random.default_rng(41)
+    T, k, E, H = 40, 6, 16, 384
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int64)
+    idx[rng.random((T, k)) < 0.15] = -1
+    lay = oracle.layout(idx, E, 4, 8)
+    rows = lay["max_rows"]
+    q = _e4m3_codes(rng, (rows, H))
+    s = np.exp2(rng.integers(-8, 9, size=(rows, H // 128))).astype(np.float32)
+    dec = torch.from_numpy(q).view(torch.float8_e4m3fn).to(torch.float32).numpy()
+    vals = dec * np.repeat(s, 128, axis=1)
+    y = bf16_bits_of(vals)
+    assert np.array_equal(f32_of_bf16(y), vals)          # exact in bf16
+    wts = rng.standard_normal((T, k)).astype(np.float32)
+    for weights in (wts, None):
+        ref, _ = oracle.combine(lay["slot_map"], T, k, y, weights)
+        got = oracle.combine_fp8(lay["slot_map"], T, k, q, s, weights)
+        assert np.array_equal(got, ref)
+
+
+def test_combine_fp8_equals_exact_rational_chain_with_general_scales():
+    # Arbitrary binary32 scales: the product decode(q) * scale rounds once
+    # to binary32, then each FMA rounds once; bf16 at the end.
+    rng = np.random.default_rng(43)
+    T, k, E, H = 8, 4, 6, 256
+    idx = rng.integers(0, E, size=(T, k)).astype(np.int64)
+    idx[rng.random((T, k)) < 0.2] = -1
+    lay = oracle.layout(idx, E, 2, 2)
+    rows = lay["max_rows"]
+    q = _e4m3_codes(rng, (rows, H))
+    s = (rng.uniform(0.5, 2.0, (rows, H // 128)) * 10.0 ** rng.integers(-3, 3, (rows, H // 128))).astype(np.float32)
+    dec = torch.from_numpy(q).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    wts = (rng.standard_normal((T, k)) * 2).astype(np.float32)
+    got = oracle.combine_fp8(lay["slot_map"], T, k, q, s, wts)
+    exp = np.empty((T, H), np.float32)
+    for t in range(T):
+        for h in range(H):
+            acc = Fraction(0)
+            for j in range(k):
+                r = lay["slot_map"][t * k + j]
+                if r < 0:
+                    continue
+                v = round_fraction(Fraction(float(dec[r, h])) * Fraction(float(s[r, h // 128])), 24)
+                acc = round_fraction(Fraction(float(wts[t, j])) * v + acc, 24)
+            exp[t, h] = float(round_fraction(acc, 8))
+    assert np.array_equal(got, bf16_bits_of(exp))
+
+
+def test_combine_fp8_of_the_fp8_dispatch_returns_the_dequantised_rows():
+    # dispatch (bf16 -> FP8) followed by the unweighted FP8 combine with one
+    # valid slot per token: each token gets back bf16(decode(q) * scale) of
+    # its own row, which is within the FP8 quantisation error of x.
+    rng = np.random.default_rng(47)
+    T, E, H = 64, 8, 256
+    idx = np.full((T, 2), -1, np.int64)
+    idx[:, 0] = rng.integers(0, E, T)
+    lay = oracle.layout(idx, E, 1, 1)
+    x = bf16_bits_of(rng.standard_normal((T, H)) * 10.0 ** rng.uniform(-2, 2, (T, 1)))
+    rq, rs = oracle.dispatch(lay, x, oracle.X_BF16_QUANT_FP8)
+    out = oracle.combine_fp8(lay["slot_map"], T, 2, rq, rs)
+    qt, st = oracle.quantize_rows(x)
+    dec = torch.from_numpy(qt).view(torch.float8_e4m3fn).to(torch.float32).numpy()
+    deq = (dec * np.repeat(st, 128, axis=1)).astype(np.float32)
+    assert np.array_equal(out, bf16_bits_of(deq))
+    xf = f32_of_bf16(x)
+    assert np.all(np.abs(f32_of_bf16(out) - xf) <= np.repeat(st, 128, axis=1) * 16 + np.abs(xf) * 2.0 ** -8)
+
+
 def test_combine_near_cancellation_equals_exact_rational_fma_chain():
     # Sums that nearly cancel: the result is tiny next to its terms, so every
     # binary32 rounding step, and the order of the steps, reaches the bf16

@@ -60,6 +60,12 @@ MUTANTS = {
                               "q[i / 2] = (uint8_t)(oracle_e2m1_encode(oracle_bf16_to_f32(x[i + 1]) * inv) |\n                             (oracle_e2m1_encode(oracle_bf16_to_f32(x[i]) * inv) << 4));"),
     "nvfp4 scale from amax / 4": ("*scale = oracle_e4m3_encode(amax / E2M1_MAX);", "*scale = oracle_e4m3_encode(amax / 4.0f);"),
     "nvfp4 divides by the unrounded scale": ("float inv = 1.0f / oracle_e4m3_decode(*scale);", "float inv = E2M1_MAX / amax;"),
+    "fp8 combine drops the scale": ("const float v = oracle_e4m3_decode(yq[(size_t)r * H + h]) * ys[(size_t)r * B + h / 128];",
+                                    "const float v = oracle_e4m3_decode(yq[(size_t)r * H + h]);"),
+    "fp8 combine takes the wrong block's scale": ("ys[(size_t)r * B + h / 128]", "ys[(size_t)r * B + h % B]"),
+    "fp8 combine sums in reverse order": ("            for (int32_t j = 0; j < k; ++j) {\n                const int32_t r = slot_map[(int64_t)t * k + j];",
+                                          "            for (int32_t j = k - 1; j >= 0; --j) {\n                const int32_t r = slot_map[(int64_t)t * k + j];"),
+    "fp8 combine rounds twice": ("sum = fmaf(wj, v, sum);", "sum = wj * v + sum;"),
     "weight gather ignores the slot map": ("(sm[j] >= 0 && recv_weights_in) ? recv_weights_in[sm[j]] : 0.0f;",
                                            "(sm[j] >= 0 && recv_weights_in) ? recv_weights_in[j] : 0.0f;"),
 }
