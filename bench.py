@@ -381,6 +381,25 @@ def run_ours(args, rank, world, dev):
                                  "gbs": round(nv_bytes / (nv_ms * 1e-3) / 1e9, 1),
                                  "frac_of_peak": round(nv_bytes / (nv_ms * 1e-3) / 1e9 / peak, 4)}
 
+    # combine of FP8 expert outputs (the dispatch's own e4m3 rows and scales stand in for them)
+    if fp8:
+        out8 = torch.empty_like(out)
+        c8 = lambda: ep.combine_fp8(recv_x, recv_s, handle, wts, out=out8)
+        for _ in range(3):
+            c8()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_f = max(3, min(50, K))
+        f0.record(stream)
+        for _ in range(n_f):
+            c8()
+        f1.record(stream)
+        torch.cuda.synchronize(dev)
+        c8_ms = f0.elapsed_time(f1) / n_f
+        c8_bytes = V * (H + (H // 128) * 4) + T * k * 8 + T * H * 2
+        res["combine_fp8"] = {"us": round(c8_ms * 1e3, 2), "bytes": c8_bytes,
+                              "gbs": round(c8_bytes / (c8_ms * 1e-3) / 1e9, 1),
+                              "frac_of_peak": round(c8_bytes / (c8_ms * 1e-3) / 1e9 / peak, 4)}
+
     # the backward of the weighted combine (training), same workload
     gy = torch.empty(rows, H, dtype=torch.bfloat16, device=dev)
     gw = torch.empty(T, k, dtype=torch.float32, device=dev)

@@ -6,11 +6,11 @@ this package is the thin Python binding.  See ``ep.py``.
 
 from .ep import (EP_DEVERR_BAD_TOPK_IDX, EP_DEVERR_CAPACITY, EP_DEVERR_TIMEOUT, EP_X_BF16,
                  EP_X_BF16_TO_FP8, EP_X_BF16_TO_NVFP4, EP_X_FP8, EPError, EPHandle, combine,
-                 combine_backward, dispatch, dispatch_mn_scales, dispatch_with_handle, get_layout, lib,
-                 library_path, max_recv_rows)
+                 combine_backward, combine_fp8, dispatch, dispatch_mn_scales, dispatch_with_handle,
+                 get_layout, lib, library_path, max_recv_rows)
 from . import mgpu
 
 __all__ = ["mgpu", "EPHandle", "EPError", "get_layout", "dispatch", "dispatch_with_handle", "combine",
-           "combine_backward", "dispatch_mn_scales",
+           "combine_backward", "combine_fp8", "dispatch_mn_scales",
            "max_recv_rows", "lib", "library_path", "EP_X_BF16", "EP_X_FP8", "EP_X_BF16_TO_FP8",
            "EP_X_BF16_TO_NVFP4", "EP_DEVERR_BAD_TOPK_IDX", "EP_DEVERR_CAPACITY", "EP_DEVERR_TIMEOUT"]

@@ -358,6 +358,33 @@ EP_API ep_status ep_combine(const ep_handle* h, const void* y, int32_t H, const 
     return ok();
 }
 
+EP_API ep_status ep_combine_fp8(const ep_handle* h, const void* y_q, const float* y_scales, int32_t H,
+                                const float* topk_weights, void* out, ep_stream_t stream) {
+    ep_status st = check_handle(h);
+    if (st != EP_OK) return st;
+    if (H < 1 || H % 128 != 0) return invalid("hidden %d must be a positive multiple of 128", H);
+    if (y_q == nullptr || !aligned(y_q, 16)) return invalid("y_q must be non-NULL and 16-byte aligned");
+    if (y_scales == nullptr || !aligned(y_scales, 4)) return invalid("y_scales must be non-NULL and 4-byte aligned");
+    if (h->num_tokens > 0 && (out == nullptr || !aligned(out, 16))) return invalid("out must be non-NULL and 16-byte aligned");
+    if (topk_weights && !aligned(topk_weights, 4)) return invalid("topk_weights misaligned");
+
+    ep::CombineFp8Args a;
+    a.y_q = y_q;
+    a.y_scales = y_scales;
+    a.topk_weights = topk_weights;
+    a.out = out;
+    a.slot_map = h->slot_map;
+    a.error_word = h->error_word;
+    a.T = h->num_tokens;
+    a.k = h->num_topk;
+    a.H = H;
+    a.max_rows = h->max_recv_rows;
+    if (a.T == 0) return ok();
+    cudaError_t err = ep::launch_combine_fp8(a, (cudaStream_t)stream);
+    if (err != cudaSuccess) return cuda_failed("combine_fp8 launch", err);
+    return ok();
+}
+
 EP_API ep_status ep_combine_backward(const ep_handle* h, const void* grad_out, const void* y, int32_t H,
                                      const float* topk_weights, void* grad_y, float* grad_weights,
                                      ep_stream_t stream) {

@@ -74,6 +74,18 @@ struct CombineArgs {
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
 
+struct CombineFp8Args {
+    const void* y_q;                 // [max_rows,H] e4m3 codes
+    const float* y_scales;           // [max_rows,H/128]
+    const float* topk_weights;       // nullable: unweighted
+    void* out;                       // [T,H] bf16
+    const int32_t* slot_map;
+    uint32_t* error_word;
+    int32_t T, k, H, max_rows;
+};
+
+cudaError_t launch_combine_fp8(const CombineFp8Args& a, cudaStream_t stream);
+
 struct CombineBackwardArgs {
     const void* grad_out;            // [T,H] bf16
     const void* y;                   // [max_rows,H] bf16

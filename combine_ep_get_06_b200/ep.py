@@ -75,6 +75,7 @@ SIGNATURES = {
                                           _P, _P, _P]),
     "ep_combine": (ctypes.c_int, [_HP, _P, _I32, _P, _P, _P, _P, _P]),
     "ep_combine_backward": (ctypes.c_int, [_HP, _P, _P, _I32, _P, _P, _P, _P]),
+    "ep_combine_fp8": (ctypes.c_int, [_HP, _P, _P, _I32, _P, _P, _P]),
     "ep_dispatch_mn_scales": (ctypes.c_int, [_HP, ctypes.c_int, _P, _P, _I32, _P, _P, _I32, _P]),
     "ep_read_recv_counts": (ctypes.c_int, [_HP, _P, _P]),
     "ep_read_total_rows": (ctypes.c_int, [_HP, ctypes.POINTER(_I32), _P]),
@@ -425,6 +426,28 @@ def combine(y: torch.Tensor, handle: EPHandle, topk_weights: Optional[torch.Tens
     _check(lib().ep_combine(handle.ref, y.data_ptr(), H, _ptr(topk_weights), _ptr(recv_topk_weights),
                             _ptr(out_w), out.data_ptr(), _stream(dev)), "combine")
     return out, out_w
+
+
+def combine_fp8(y_q: torch.Tensor, y_scales: torch.Tensor, handle: EPHandle,
+                topk_weights: Optional[torch.Tensor] = None, *, out: Optional[torch.Tensor] = None):
+    """Combine of FP8 expert outputs: y_q [max_recv_rows, H] e4m3 (or uint8)
+    codes with y_scales [max_recv_rows, H/128] f32, in the layout of the FP8
+    dispatch's output.  Each value is decode(q) * scale (binary32), summed
+    like combine.  -> out [T, H] bf16."""
+    dev = handle.device
+    _need(y_q, "y_q", (torch.float8_e4m3fn, torch.uint8), dev, 2)
+    _need(y_scales, "y_scales", (torch.float32,), dev, 2)
+    rows, H = y_q.shape
+    if rows != handle.max_recv_rows or tuple(y_scales.shape) != (rows, H // 128):
+        raise ValueError("y_q must be [max_recv_rows, hidden] and y_scales [max_recv_rows, hidden/128]")
+    if topk_weights is not None:
+        _need(topk_weights, "topk_weights", (torch.float32,), dev, 2)
+    if out is None:
+        out = torch.empty(handle.num_tokens, H, dtype=torch.bfloat16, device=dev)
+    _need(out, "out", (torch.bfloat16,), dev, 2)
+    _check(lib().ep_combine_fp8(handle.ref, y_q.data_ptr(), y_scales.data_ptr(), H, _ptr(topk_weights),
+                                out.data_ptr(), _stream(dev)), "combine_fp8")
+    return out
 
 
 def combine_backward(grad_out: torch.Tensor, y: torch.Tensor, handle: EPHandle,

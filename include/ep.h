@@ -239,6 +239,21 @@ EP_API ep_status ep_combine(const ep_handle* handle, const void* y, int32_t hidd
                             const float* topk_weights, const float* recv_weights_in,
                             float* out_weights, void* out, ep_stream_t stream);
 
+/* Combine of FP8 expert outputs: the low-precision combine (the DeepEP V2
+ * README's introduction says its kernels support low precision, FP8
+ * included; it fixes no arithmetic, so this is the plainest reading).  The
+ * expert outputs come in the layout of the FP8 dispatch's output:
+ *   y_q      [max_recv_rows,H] e4m3 codes (16-byte aligned)
+ *   y_scales [max_recv_rows,H/128] f32, one scale per 1x128 block
+ * Each value is v = decode(q) * scale in binary32 (one rounding), and
+ *   out[t,:] = bf16( sum_j w[t,j] * v[slot_map[t*k+j],:] )
+ * with the accumulation of ep_combine (fp32 FMA from +0 in ascending j, one
+ * bf16 rounding).  topk_weights [T,k] f32 or NULL (every w = 1); out [T,H]
+ * bf16.  H % 128 == 0.  Only rows of valid slots are read. */
+EP_API ep_status ep_combine_fp8(const ep_handle* handle, const void* y_q, const float* y_scales,
+                                int32_t hidden, const float* topk_weights, void* out,
+                                ep_stream_t stream);
+
 /* Backward of the weighted combine (combine_backward of the DeepEP V2
  * README, "Interfaces and examples", which runs as a dispatch of the output
  * gradient; with weights in the forward each row is also scaled):
