@@ -433,6 +433,22 @@ def _e4m3_codes(rng, shape):
     return c | (rng.integers(0, 2, size=shape).astype(np.uint8) << 7)
 
 
+def test_combine_fp8_hand_derived_examples(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "combine_fp8_hand_example.json")))
+    H = g["H"]
+    for case in g["cases"]:
+        k = len(case["codes"])
+        q = np.zeros((k, H), np.uint8)
+        q[:, 0] = [c[0] for c in case["codes"]]
+        s = np.array(case["scales"], np.float32).reshape(k, 1)
+        sm = np.arange(k, dtype=np.int32)
+        if case.get("drop_second"):
+            sm[1] = -1
+        out = oracle.combine_fp8(sm, 1, k, q, s, np.array([case["weights"]], np.float32))
+        assert int(out[0, 0]) == case["out_bf16"], case["note"]
+        assert np.all(out[0, 1:] == 0)
+
+
 def test_combine_fp8_with_power_of_two_scales_is_the_bf16_combine_of_the_decoded_values():
     # With a power-of-two scale, decode(q) * scale is exact and fits bf16
     # (3 mantissa bits in 7), so the FP8 combine must equal the bf16 combine
