@@ -45,8 +45,8 @@
  * on another GPU: the ordering across ranks comes from the caller's
  * collectives in steps 2, 4 and 6.  Nothing in this file has been run
  * across several GPUs.  Its kernels were checked with all W blocks on one
- * GPU, and the whole path (CUDA IPC included) with two processes sharing
- * one GPU.  The stores over NVLink have not run.
+ * GPU, and the whole path (CUDA IPC included) with two and four processes
+ * sharing one GPU.  The stores over NVLink have not run.
  */
 #ifndef EP_B200_EP_MULTI_H
 #define EP_B200_EP_MULTI_H

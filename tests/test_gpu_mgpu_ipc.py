@@ -1,9 +1,9 @@
 """The multi-process expert-parallel path on one GPU, through real CUDA IPC.
 
-Two processes share GPU 0, one per rank.  Each allocates its rank block
-with the library (cudaMalloc) and exports it.  The other process maps it
+Two or four processes share GPU 0, one per rank.  Each allocates its rank block
+with the library (cudaMalloc) and exports it.  Every other process maps it
 (cudaIpcOpenMemHandle), and the dispatch and combine kernels store into
-and load from the peer's block.  The ranks' kernels never wait on one
+and load from the peers' blocks.  The ranks' kernels never wait on one
 another: each step's ordering comes from the host, where every collective
 first synchronises the rank's stream and then meets the other rank over
 gloo.  Each rank checks its own block and its combine output bit for bit
@@ -59,7 +59,7 @@ def _rank_main(rank, world, port, out):
         from combine_ep_get_06_b200 import mgpu
 
         w = W.WORKLOADS["mid"]
-        Ts = [700, 512]
+        Ts = [700, 512, 300, 640][:world]
         Tmax, E, k, a, H = 1024, w.E, w.k, w.align, w.H
         epr = E // world
         inps = [W.make_inputs(w, seed=80 + r, T=Ts[r]) for r in range(world)]
@@ -124,10 +124,10 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def test_two_processes_share_blocks_through_cuda_ipc():
+@pytest.mark.parametrize("world", [2, 4])
+def test_processes_share_blocks_through_cuda_ipc(world):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-    world = 2
     manager = mp.get_context("spawn").Manager()
     out = manager.dict()
     try:
