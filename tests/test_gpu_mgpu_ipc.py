@@ -5,7 +5,7 @@ with the library (cudaMalloc) and exports it.  Every other process maps it
 (cudaIpcOpenMemHandle), and the dispatch and combine kernels store into
 and load from the peers' blocks.  The ranks' kernels never wait on one
 another: each step's ordering comes from the host, where every collective
-first synchronises the rank's stream and then meets the other rank over
+first synchronises the rank's stream and then meets the other ranks over
 gloo.  Each rank checks its own block and its combine output bit for bit
 against the oracle's one-GPU layout of the concatenated batch, then the
 group unmaps and frees."""
