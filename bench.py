@@ -69,6 +69,9 @@ def parse_args():
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-mgpu", action="store_true")
+    p.add_argument("--ep", action="store_true",
+                   help="time the expert-parallel group across the torchrun ranks (one GPU each) instead of "
+                        "the one-GPU step")
     return p.parse_args()
 
 
@@ -213,6 +216,74 @@ def combine_traffic(workload: str, T: int):
 
 
 # ------------------------------------------------------------- our arm
+
+def run_ep(args, rank, world, dev):
+    """Expert parallelism across the ranks (segments = ranks, one GPU each):
+    each rank routes its own V3-shaped batch; ExpertParallelGroup.dispatch
+    (layout, all-gather of counts, dispatch kernel storing into the owners'
+    blocks over NVLink, barrier) then .combine (barrier, combine kernel
+    loading from them).  Reported like the pages' logical bandwidth: the
+    rows a rank sends (or pulls back), local ones included, over the time,
+    summed over ranks, max time over ranks."""
+    import torch
+    import torch.distributed as dist
+
+    import combine_ep_get_06_b200 as ep
+    from combine_ep_get_06_b200 import mgpu
+
+    w = W.WORKLOADS[args.workload]
+    T = args.tokens if args.tokens is not None else w.T
+    inp = W.make_inputs(w, seed=rank, T=T)
+    x = torch.from_numpy(np.ascontiguousarray(inp["x"]).view(np.int16)).view(torch.bfloat16).to(dev)
+    idx = torch.from_numpy(inp["topk_idx"]).to(dev)
+    wts = torch.from_numpy(inp["topk_weights"]).to(dev)
+    fp8 = w.x_mode == "fp8_quant"
+    grp = mgpu.ExpertParallelGroup(T, w.k, w.E, w.H, expert_alignment=w.align,
+                                   mode=ep.EP_X_BF16_TO_FP8 if fp8 else ep.EP_X_BF16, device=dev)
+    try:
+        grp.block.y.zero_()                      # stands in for the expert GEMMs' output
+        out = torch.empty(T, w.H, dtype=torch.bfloat16, device=dev)
+        for _ in range(args.warmup):
+            h = grp.dispatch(x, idx, wts, use_fp8=fp8)
+            grp.combine(h, wts, out)
+        torch.cuda.synchronize(dev)
+        stream = torch.cuda.current_stream(dev)
+        K = args.steps
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        for i in range(K):
+            ev[i][0].record(stream)
+            h = grp.dispatch(x, idx, wts, use_fp8=fp8)
+            ev[i][1].record(stream)
+            grp.combine(h, wts, out)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize(dev)
+        d_ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in ev), world, dev)
+        c_ms = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in ev), world, dev)
+        grp.kernels.check_error()
+        V = int((idx >= 0).sum().item())
+        row = w.H + (w.H // 128) * 4 if fp8 else 2 * w.H
+        d_bytes = V * row * world                # rows sent by all ranks
+        c_bytes = V * w.H * 2 * world            # rows pulled back by all ranks
+        res = {"metric": "expert-parallel dispatch & combine logical GB/s across ranks (V3 shape)",
+               "value": round((d_bytes + c_bytes) / ((d_ms + c_ms) * 1e-3) / 1e9, 2), "unit": "GB/s",
+               "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(d_ms + c_ms, 5),
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+               "dtype": "f32", "data": "synthetic",
+               "config": {**step_config(w, T, world), "parallelism": f"ep{world}"},
+               "dispatch": {"us": round(d_ms * 1e3, 2),
+                            "logical_gbs_per_rank": round(d_bytes / world / (d_ms * 1e-3) / 1e9, 1),
+                            "includes": "layout, all-gather of counts, dispatch kernel, barrier"},
+               "combine": {"us": round(c_ms * 1e3, 2),
+                           "logical_gbs_per_rank": round(c_bytes / world / (c_ms * 1e-3) / 1e9, 1),
+                           "includes": "barrier, combine kernel"},
+               "pages_sm100_nvlink_context": {"dispatch_gbs": 726, "combine_gbs": 740, "sms": 64}}
+    finally:
+        grp.close()
+    return res
+
 
 def run_ours(args, rank, world, dev):
     import torch
@@ -760,7 +831,7 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
     try:
-        res = run_ours(args, rank, world, dev)
+        res = run_ep(args, rank, world, dev) if args.ep else run_ours(args, rank, world, dev)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

@@ -299,6 +299,28 @@ class _TorchComm:
         self.dist.all_reduce(self._word, group=self.group)
 
 
+class _SingleRank:
+    """The collectives of a group of one rank (no process group)."""
+
+    rank, world = 0, 1
+
+    def all_gather_objects(self, obj) -> list:
+        return [obj]
+
+    def all_gather_counts(self, out: torch.Tensor, inp: torch.Tensor):
+        out[0].copy_(inp)
+
+    def barrier(self, device):
+        pass
+
+
+def _default_comm(group):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        return _TorchComm(group)
+    return _SingleRank()
+
+
 class _CudaIpc:
     """Block allocation and CUDA IPC through the library."""
 
@@ -328,12 +350,13 @@ class ExpertParallelGroup:
 
     Every rank must make the same calls in the same order (each one holds
     collectives).  ``comm``, ``ipc`` and ``kernels`` default to
-    torch.distributed, CUDA IPC and this library; tests pass host fakes."""
+    torch.distributed (a group of one rank when no process group is
+    initialised), CUDA IPC and this library; tests pass host fakes."""
 
     def __init__(self, max_tokens: int, num_topk: int, num_experts: int, hidden: int, *,
                  expert_alignment: int = 1, mode: int = EP_X_BF16_TO_FP8, group=None, device=None,
                  comm=None, ipc=None, kernels=None):
-        self.comm = comm if comm is not None else _TorchComm(group)
+        self.comm = comm if comm is not None else _default_comm(group)
         self.ipc = ipc if ipc is not None else _CudaIpc()
         self.rank, self.world = self.comm.rank, self.comm.world
         self.device = torch.device(device) if device is not None else torch.device(
