@@ -12,15 +12,22 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "ep_oracle.c")
 LIB = os.path.join(HERE, "_ep_oracle.so")
+SELFTEST = os.path.join(HERE, "selftest.c")
+FLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-Wall", "-Wextra"]
 
 
 def compile_to(src: str, out: str) -> str:
     """Compiles an oracle source file with the oracle's flags."""
     tmp = out + f".tmp{os.getpid()}"
-    cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
-           "-fvisibility=hidden", "-Wall", "-Wextra", "-o", tmp, src, "-lm"]
+    cmd = ["gcc", *FLAGS, "-fPIC", "-shared", "-fvisibility=hidden", "-o", tmp, src, "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, out)
+    return out
+
+
+def compile_selftest(out: str) -> str:
+    """The oracle's C self-test (hand-derived values) as an executable."""
+    subprocess.run(["gcc", *FLAGS, "-Werror", "-o", out, SELFTEST, "-lm"], check=True)
     return out
 
 
