@@ -226,6 +226,27 @@ def test_quantize_hand_example():
     assert s[0, 0] == np.float32(2.0) / np.float32(448.0)
 
 
+def test_quantize_product_form_golden(golden_dir):
+    # Two blocks whose scaled value is exactly the e4m3 midpoint 336, derived
+    # by hand: q = e4m3(RN(x * RN(448/amax))) rounds block 0 up and lands
+    # block 1 on the tie, while q = e4m3(RN(x / RN(amax/448))) does the
+    # opposite, so the two readings give different codes in both blocks.
+    g = json.load(open(os.path.join(golden_dir, "fp8_quant_product_form.json")))
+    H = g["hidden"]
+    x = np.zeros((1, H), np.float32)
+    for b, vals in enumerate(g["x"]):
+        x[0, b * 128:b * 128 + len(vals)] = vals
+    xb = bf16_bits_of(x)
+    assert np.array_equal(f32_of_bf16(xb), x)          # every input is bf16-exact
+    q, s = oracle.quantize_rows(xb)
+    for b, codes in enumerate(g["codes"]):
+        blk = q[0, b * 128:(b + 1) * 128]
+        assert list(blk[:len(codes)]) == codes
+        assert np.all(blk[len(codes):] == 0)
+        m, e = g["scales_exact"][b]
+        assert Fraction(float(s[0, b])) == Fraction(m) * Fraction(2) ** e
+
+
 def test_quantize_invariants():
     rng = np.random.default_rng(3)
     H = 1024

@@ -28,6 +28,8 @@ MUTANTS = {
     "e4m3 sign dropped": ("uint8_t sign = signbit(v) ? 0x80 : 0x00;", "uint8_t sign = 0x00;"),
     "amax floor dropped": ("if (amax < AMAX_FLOOR) amax = AMAX_FLOOR;", ""),
     "scale transposed": ("*scale = amax / E4M3_MAX;", "*scale = E4M3_MAX / amax;"),
+    "quantise divides by the scale": ("for (int i = 0; i < QBLOCK; ++i) q[i] = oracle_e4m3_encode(oracle_bf16_to_f32(x[i]) * inv);",
+                                      "for (int i = 0; i < QBLOCK; ++i) q[i] = oracle_e4m3_encode(oracle_bf16_to_f32(x[i]) / *scale);"),
     "amax misses last value": ("for (int i = 0; i < QBLOCK; ++i) amax = fmaxf",
                                "for (int i = 0; i < QBLOCK - 1; ++i) amax = fmaxf"),
     "alignment rounds up one block too many": ("int32_t padded = (counts[e] + align - 1) / align * align;",
