@@ -33,7 +33,6 @@ import datetime
 import hashlib
 import json
 import os
-import re
 import statistics
 import subprocess
 import sys
@@ -51,6 +50,7 @@ METRIC = "dispatch & combine GB/s and % of B200 HBM peak (V3 shape); decode µs/
 WORKLOAD = "v3"
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0   # the nominal HBM3e figure the target is stated against
+DTYPE = "bf16->e4m3 (1x128 scales), f32 accumulation"   # what the path computes in
 
 
 def parse_args():
@@ -69,6 +69,8 @@ def parse_args():
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-mgpu", action="store_true")
+    p.add_argument("--no-extra-workloads", action="store_true",
+                   help="skip the mid and skewed lines")
     p.add_argument("--ep", action="store_true",
                    help="time the expert-parallel group across the torchrun ranks (one GPU each) instead of "
                         "the one-GPU step")
@@ -196,26 +198,36 @@ def nvsmi_device_id(dev) -> str | None:
 
 def combine_traffic(workload: str, T: int):
     """Per-launch DRAM bytes of the combine kernel from the committed ncu
-    summary, if that summary was taken on the current combine source and
-    on this workload."""
+    record (profiles/traffic.json), if that record was taken on the current
+    combine source and on this workload; else None."""
     src = os.path.join(ROOT, "combine_ep_get_06_b200", "csrc", "combine.cu")
-    summ = os.path.join(ROOT, "profiles", "combine_kernel_v3.md")
+    rec = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        text = open(summ).read()
-    except OSError:
+        r = json.load(open(rec))["combine_kernel"]
+    except (OSError, ValueError, KeyError):
         return None
-    m_sha = re.search(r"combine\.cu sha256\[:16\]:\s*`?([0-9a-f]{16})", text)
-    m_tr = re.search(r"traffic per launch \(bytes\):\s*([0-9]+)", text)
-    m_wl = re.search(r"profiled workload:\s*(\w+) T=([0-9]+)", text)
-    if not (m_wl and m_wl.group(1) == workload and int(m_wl.group(2)) == T):
+    if r.get("workload") != workload or int(r.get("T", -1)) != T or r.get("source_sha16") != sha:
         return None
-    if m_sha and m_tr and m_sha.group(1) == sha:
-        return int(m_tr.group(1))
-    return None
+    return int(r["dram_read_bytes"]) + int(r["dram_write_bytes"])
 
 
 # ------------------------------------------------------------- our arm
+
+def time_back_to_back(fn, n: int, stream) -> float:
+    """Mean ms per call of n back-to-back calls of fn on `stream` (CUDA events), after 3 untimed ones."""
+    import torch
+
+    for _ in range(3):
+        fn()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        fn()
+    b.record(stream)
+    b.synchronize()
+    return a.elapsed_time(b) / n
+
 
 def run_ep(args, rank, world, dev):
     """Expert parallelism across the ranks (segments = ranks, one GPU each):
@@ -263,15 +275,19 @@ def run_ep(args, rank, world, dev):
         d_ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in ev), world, dev)
         c_ms = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in ev), world, dev)
         grp.kernels.check_error()
-        V = int((idx >= 0).sum().item())
+        # valid slots summed over the ranks (each rank routes its own batch)
+        V = (idx >= 0).sum().to(torch.int64).reshape(1)
+        if world > 1:
+            dist.all_reduce(V)
+        V = int(V.item())
         row = w.H + (w.H // 128) * 4 if fp8 else 2 * w.H
-        d_bytes = V * row * world                # rows sent by all ranks
-        c_bytes = V * w.H * 2 * world            # rows pulled back by all ranks
+        d_bytes = V * row                        # rows sent by all ranks
+        c_bytes = V * w.H * 2                    # rows pulled back by all ranks
         res = {"metric": "expert-parallel dispatch & combine logical GB/s across ranks (V3 shape)",
                "value": round((d_bytes + c_bytes) / ((d_ms + c_ms) * 1e-3) / 1e9, 2), "unit": "GB/s",
                "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(d_ms + c_ms, 5),
                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-               "dtype": "f32", "data": "synthetic",
+               "dtype": DTYPE, "data": "synthetic",
                "config": {**step_config(w, T, world), "parallelism": f"ep{world}"},
                "dispatch": {"us": round(d_ms * 1e3, 2),
                             "logical_gbs_per_rank": round(d_bytes / world / (d_ms * 1e-3) / 1e9, 1),
@@ -326,11 +342,16 @@ def run_ours(args, rank, world, dev):
     def dispatch():
         ep.dispatch_with_handle(x, handle, use_fp8=fp8, recv_x=recv_x, recv_scales=recv_s)
 
+    def layout_dispatch():   # the pages' dispatch(x, topk_idx, ...): routes and sends in one call
+        ep.dispatch(x, idx, wts, w.E, expert_alignment=w.align, num_segments=w.S, handle=handle,
+                    use_fp8=fp8, recv_x=recv_x, recv_scales=recv_s, recv_topk_idx=recv_idx,
+                    recv_topk_weights=recv_w)
+
     def combine():
         ep.combine(y, handle, wts, out=out)
 
     for _ in range(args.warmup):
-        layout(); dispatch(); combine()
+        layout_dispatch(); combine()
     torch.cuda.synchronize(dev)
     V = int(handle.counts.sum())
     P = int(handle.num_pad_rows[0])
@@ -339,7 +360,7 @@ def run_ours(args, rank, world, dev):
     handle.check_error()
 
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(nvsmi_device_id(dev))
     if world > 1:
@@ -350,19 +371,17 @@ def run_ours(args, rank, world, dev):
     start.record(stream)
     for i in range(K):
         e = ev[i]
-        e[0].record(stream); layout()
-        e[1].record(stream); dispatch()
-        e[2].record(stream); combine()
-        e[3].record(stream)
+        e[0].record(stream); layout_dispatch()
+        e[1].record(stream); combine()
+        e[2].record(stream)
     end.record(stream)
     torch.cuda.synchronize(dev)
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
     total_ms = start.elapsed_time(end)
-    lay_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
-    dis_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
-    com_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+    ld_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    com_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
     handle.check_error()
 
     total_ms = max_over_ranks(total_ms, world, dev)
@@ -371,22 +390,43 @@ def run_ours(args, rank, world, dev):
     value = weak_scaling_gbs(step_total, world, ms_per_step)
     peak, peak_kind = hbm_peak()
 
+    # the same step as two calls (layout, then dispatch with the handle), and
+    # the dispatch kernel alone back to back, both after the timed region
+    K2 = max(5, min(50, K))
+    ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K2)]
+    for i in range(K2):
+        e = ev2[i]
+        e[0].record(stream); layout()
+        e[1].record(stream); dispatch()
+        e[2].record(stream); combine()
+        e[3].record(stream)
+    torch.cuda.synchronize(dev)
+    lay_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev2)
+    two_dis_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev2)
+    two_step_ms = statistics.mean(e[0].elapsed_time(e[3]) for e in ev2)
+    dis_ms = time_back_to_back(dispatch, K2, stream)
+    handle.check_error()
+
+    def rate(nb, ms):
+        gbs = nb / (ms * 1e-3) / 1e9
+        return {"us": round(ms * 1e3, 2), "bytes": nb, "gbs": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4),
+                "frac_of_nominal_8tbs": round(gbs / NOMINAL_HBM_GBS, 4)}
+
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": DTYPE, "data": "synthetic",
         "config": step_config(w, T, world),
         "gpu_launches": K * (layout_launches(T, k) + 2),
-        "layout_us": round(lay_ms * 1e3, 2),
-        "dispatch": {"us": round(dis_ms * 1e3, 2), "bytes": nbytes["dispatch"],
-                     "gbs": round(nbytes["dispatch"] / (dis_ms * 1e-3) / 1e9, 1),
-                     "frac_of_peak": round(nbytes["dispatch"] / (dis_ms * 1e-3) / 1e9 / peak, 4),
-                     "frac_of_nominal_8tbs": round(nbytes["dispatch"] / (dis_ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 4),
-                     "valid_rows": V, "padding_rows": P},
-        "combine": {"us": round(com_ms * 1e3, 2), "bytes": nbytes["combine"],
-                    "gbs": round(nbytes["combine"] / (com_ms * 1e-3) / 1e9, 1),
-                    "frac_of_peak": round(nbytes["combine"] / (com_ms * 1e-3) / 1e9 / peak, 4),
-                    "frac_of_nominal_8tbs": round(nbytes["combine"] / (com_ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 4)},
+        "step": "ep_layout_dispatch (layout + FP8 dispatch, one call) -> ep_combine",
+        "layout_dispatch": {**rate(nbytes["layout"] + nbytes["dispatch"], ld_ms),
+                            "note": "in the timed step: layout kernels and the dispatch kernel of one call"},
+        "combine": rate(nbytes["combine"], com_ms),
+        "dispatch": {**rate(nbytes["dispatch"], dis_ms), "valid_rows": V, "padding_rows": P,
+                     "note": "the dispatch kernel alone, back to back after the timed step"},
+        "two_call": {"layout_us": round(lay_ms * 1e3, 2), "dispatch_us": round(two_dis_ms * 1e3, 2),
+                     "step_us": round(two_step_ms * 1e3, 2),
+                     "note": "ep_get_layout, ep_dispatch, ep_combine as separate calls"},
         "clocks": clocks,
     }
     achieved = nbytes["combine"] / (com_ms * 1e-3) / 1e9
@@ -395,103 +435,42 @@ def run_ours(args, rank, world, dev):
                        "frac": round(achieved / peak, 4), "traffic": combine_traffic(w.name, T),
                        "algorithmic_bytes": nbytes["combine"]}
 
+    n_x = max(5, min(50, K))
+
     # FP8 dispatch with GEMM-ready (MN-major) scales, same workload
     if fp8:
         ld = (rows + 3) // 4 * 4
         sc_mn = torch.empty(H // 128, ld, dtype=torch.float32, device=dev)
         mn = lambda: ep.dispatch_mn_scales(x, handle, recv_x=recv_x, recv_scales_mn=sc_mn, scales_ld=ld)
-        for _ in range(3):
-            mn()
-        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n_m = max(3, min(50, K))
-        m0.record(stream)
-        for _ in range(n_m):
-            mn()
-        m1.record(stream)
-        torch.cuda.synchronize(dev)
-        mn_ms = m0.elapsed_time(m1) / n_m
-        res["dispatch_mn_scales"] = {"us": round(mn_ms * 1e3, 2), "bytes": nbytes["dispatch"],
-                                     "gbs": round(nbytes["dispatch"] / (mn_ms * 1e-3) / 1e9, 1),
-                                     "frac_of_peak": round(nbytes["dispatch"] / (mn_ms * 1e-3) / 1e9 / peak, 4)}
-
-    # layout + dispatch in one call (ep_layout_dispatch), same workload
-    one = lambda: ep.dispatch(x, idx, wts, w.E, expert_alignment=w.align, num_segments=w.S, handle=handle,
-                              use_fp8=fp8, recv_x=recv_x, recv_scales=recv_s, recv_topk_idx=recv_idx,
-                              recv_topk_weights=recv_w)
-    for _ in range(3):
-        one()
-    o0, o1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    n_o = max(3, min(50, K))
-    o0.record(stream)
-    for _ in range(n_o):
-        one()
-    o1.record(stream)
-    torch.cuda.synchronize(dev)
-    one_ms = o0.elapsed_time(o1) / n_o
-    res["layout_dispatch_one_call"] = {"us": round(one_ms * 1e3, 2),
-                                       "bytes": nbytes["layout"] + nbytes["dispatch"],
-                                       "gbs": round((nbytes["layout"] + nbytes["dispatch"]) / (one_ms * 1e-3) / 1e9, 1)}
+        res["dispatch_mn_scales"] = rate(nbytes["dispatch"], time_back_to_back(mn, n_x, stream))
 
     # NVFP4 dispatch (E2M1 codes, one e4m3 scale per 1x16 block), same workload
     if H % 32 == 0:
         nv_x = torch.empty(rows, H // 2, dtype=torch.uint8, device=dev)
         nv_s = torch.empty(rows, H // 16, dtype=torch.uint8, device=dev)
         nv = lambda: ep.dispatch_with_handle(x, handle, use_nvfp4=True, recv_x=nv_x, recv_scales=nv_s)
-        for _ in range(3):
-            nv()
-        n0, n1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n_n = max(3, min(50, K))
-        n0.record(stream)
-        for _ in range(n_n):
-            nv()
-        n1.record(stream)
-        torch.cuda.synchronize(dev)
-        nv_ms = n0.elapsed_time(n1) / n_n
         nv_bytes = T * H * 2 + T * k * 4 + (V + P) * (H // 2 + H // 16)
-        res["dispatch_nvfp4"] = {"us": round(nv_ms * 1e3, 2), "bytes": nv_bytes,
-                                 "gbs": round(nv_bytes / (nv_ms * 1e-3) / 1e9, 1),
-                                 "frac_of_peak": round(nv_bytes / (nv_ms * 1e-3) / 1e9 / peak, 4)}
+        res["dispatch_nvfp4"] = rate(nv_bytes, time_back_to_back(nv, n_x, stream))
 
     # combine of FP8 expert outputs (the dispatch's own e4m3 rows and scales stand in for them)
     if fp8:
         out8 = torch.empty_like(out)
         c8 = lambda: ep.combine_fp8(recv_x, recv_s, handle, wts, out=out8)
-        for _ in range(3):
-            c8()
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n_f = max(3, min(50, K))
-        f0.record(stream)
-        for _ in range(n_f):
-            c8()
-        f1.record(stream)
-        torch.cuda.synchronize(dev)
-        c8_ms = f0.elapsed_time(f1) / n_f
         c8_bytes = V * (H + (H // 128) * 4) + T * k * 8 + T * H * 2
-        res["combine_fp8"] = {"us": round(c8_ms * 1e3, 2), "bytes": c8_bytes,
-                              "gbs": round(c8_bytes / (c8_ms * 1e-3) / 1e9, 1),
-                              "frac_of_peak": round(c8_bytes / (c8_ms * 1e-3) / 1e9 / peak, 4)}
+        res["combine_fp8"] = rate(c8_bytes, time_back_to_back(c8, n_x, stream))
 
     # the backward of the weighted combine (training), same workload
     gy = torch.empty(rows, H, dtype=torch.bfloat16, device=dev)
     gw = torch.empty(T, k, dtype=torch.float32, device=dev)
     g_out = out  # any [T,H] bf16 gradient; the forward's output serves
     bwd = lambda: ep.combine_backward(g_out, y, handle, wts, grad_y=gy, grad_weights=gw)
-    for _ in range(3):
-        bwd()
-    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    n_b = max(3, min(50, K))
-    b0.record(stream)
-    for _ in range(n_b):
-        bwd()
-    b1.record(stream)
-    torch.cuda.synchronize(dev)
-    bwd_ms = b0.elapsed_time(b1) / n_b
     bwd_bytes = T * H * 2 + V * H * 2 + (V + P) * H * 2 + T * k * 12
-    res["combine_backward"] = {"us": round(bwd_ms * 1e3, 2), "bytes": bwd_bytes,
-                               "gbs": round(bwd_bytes / (bwd_ms * 1e-3) / 1e9, 1),
-                               "frac_of_peak": round(bwd_bytes / (bwd_ms * 1e-3) / 1e9 / peak, 4)}
+    res["combine_backward"] = rate(bwd_bytes, time_back_to_back(bwd, n_x, stream))
     handle.check_error()
 
+    if not args.no_extra_workloads and args.tokens is None and w.name == WORKLOAD:
+        for name in ("mid", "skewed"):
+            res[name] = run_workload_lines(args, dev, name, peak)
     if not args.no_mgpu and H % 128 == 0:
         res["mgpu_local"] = run_mgpu_local(args, dev, w, inp, nbytes)
     if not args.no_decode:
@@ -501,6 +480,54 @@ def run_ours(args, rank, world, dev):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w, inp, y_np)
     return res
+
+
+def run_workload_lines(args, dev, name: str, peak: float) -> dict:
+    """Dispatch and combine GB/s on another workload (its own seeded inputs):
+    the step (one-call layout + dispatch, then combine) per call, and the
+    dispatch and combine kernels alone, back to back."""
+    import torch
+
+    import combine_ep_get_06_b200 as ep
+
+    w = W.WORKLOADS[name]
+    inp = W.make_inputs(w, seed=0)
+    T, k, H = w.T, w.k, w.H
+
+    def bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    x = bf16(inp["x"])
+    y = bf16(W.make_y(w, seed=0))
+    idx = torch.from_numpy(inp["topk_idx"]).to(dev)
+    wts = torch.from_numpy(inp["topk_weights"]).to(dev)
+    fp8 = w.x_mode == "fp8_quant"
+    handle = ep.EPHandle(T, k, w.E, w.S, w.align, device=dev)
+    rows = handle.max_recv_rows
+    recv_x = torch.empty(rows, H, dtype=torch.float8_e4m3fn if fp8 else torch.bfloat16, device=dev)
+    recv_s = torch.empty(rows, H // 128, dtype=torch.float32, device=dev) if fp8 else None
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    one = lambda: ep.dispatch(x, idx, wts, w.E, expert_alignment=w.align, num_segments=w.S, handle=handle,
+                              use_fp8=fp8, recv_x=recv_x, recv_scales=recv_s)
+    dis = lambda: ep.dispatch_with_handle(x, handle, use_fp8=fp8, recv_x=recv_x, recv_scales=recv_s)
+    com = lambda: ep.combine(y, handle, wts, out=out)
+    n = max(5, min(50, args.steps))
+    step_ms = time_back_to_back(lambda: (one(), com()), n, stream)
+    dis_ms = time_back_to_back(dis, n, stream)
+    com_ms = time_back_to_back(com, n, stream)
+    handle.check_error()
+    V = int(handle.counts.sum())
+    P = int(handle.num_pad_rows[0])
+    nb = step_bytes(w, T, V, P, handle.total_rows())
+
+    def line(b, ms):
+        gbs = b / (ms * 1e-3) / 1e9
+        return {"us": round(ms * 1e3, 2), "bytes": b, "gbs": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4)}
+
+    return {"config": step_config(w, T, 1)["workload"], "valid_rows": V, "padding_rows": P,
+            "step": line(sum(nb.values()), step_ms), "dispatch": line(nb["dispatch"], dis_ms),
+            "combine": line(nb["combine"], com_ms)}
 
 
 def run_mgpu_local(args, dev, w, inp, nbytes, world=8):
@@ -696,9 +723,8 @@ def run_e2e(args, dev, w, inp, y_np, nbytes):
             s_k.wait_event(d["in_done"])
             if i >= 2:
                 s_k.wait_event(d["out_done"])         # its outputs have been copied out
-            ep.get_layout(d["i"], w.E, num_segments=w.S, expert_alignment=w.align, topk_weights=d["w"],
-                          handle=d["handle"])
-            ep.dispatch_with_handle(d["x"], d["handle"], use_fp8=fp8, recv_x=d["rq"], recv_scales=d["rs"])
+            ep.dispatch(d["x"], d["i"], d["w"], w.E, expert_alignment=w.align, num_segments=w.S,
+                        handle=d["handle"], use_fp8=fp8, recv_x=d["rq"], recv_scales=d["rs"])
             d["disp_done"].record(s_k)
             ep.combine(d["y"], d["handle"], d["w"], out=d["out"])
             d["comp_done"].record(s_k)
@@ -803,9 +829,9 @@ def run_reference(args):
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_t / args.steps * 1e3, 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": DTYPE,
         "data": "synthetic",
-        "config": step_config(w, w.T, world),
+        "config": {**step_config(w, T_s, world), "sampled_from": f"{w.name} T={w.T}"},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -14,12 +14,15 @@
 // host it only stands for the symbol), so the first call on each device
 // looks up its device address with cudaGetSymbolAddress, with that device
 // current, and keeps it; that first call should therefore come before any
-// stream capture.  All calls share the one array: calls whose layouts
+// stream capture.  The address is kept for the life of the process: a
+// cudaDeviceReset of that device after the first call makes it stale, and
+// is not supported.  All calls share the one array: calls whose layouts
 // overlap on the GPU (other streams, or other threads on the same device)
 // race on it.  Nothing in it needs to start at zero: every entry the
 // layout reads is written earlier by the same call.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "ep_internal.h"
@@ -30,22 +33,26 @@ static __device__ __align__(256) unsigned char g_layout_scratch[EP_STATIC_LAYOUT
 
 constexpr int kMaxDevices = 128;
 std::mutex g_setup_mutex;
-void* g_scratch_ptr[kMaxDevices];  // device address of g_layout_scratch, per device
+std::atomic<void*> g_scratch_ptr[kMaxDevices];  // device address of g_layout_scratch, per device
 
-// The device address of the scratch array on the current device.
+// The device address of the scratch array on the current device: looked up
+// once per device (under a lock), then read without one.
 cudaError_t scratch_on_current_device(void** out) {
     int dev = -1;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (g_scratch_ptr[dev] == nullptr) {
-        void* p = nullptr;
-        err = cudaGetSymbolAddress(&p, g_layout_scratch);
-        if (err != cudaSuccess) return err;
-        g_scratch_ptr[dev] = p;
+    void* p = g_scratch_ptr[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
+        std::lock_guard<std::mutex> lock(g_setup_mutex);
+        p = g_scratch_ptr[dev].load(std::memory_order_relaxed);
+        if (p == nullptr) {
+            err = cudaGetSymbolAddress(&p, g_layout_scratch);
+            if (err != cudaSuccess) return err;
+            g_scratch_ptr[dev].store(p, std::memory_order_release);
+        }
     }
-    *out = g_scratch_ptr[dev];
+    *out = p;
     return cudaSuccess;
 }
 

@@ -102,7 +102,8 @@ typedef struct ep_handle {
     uint32_t* error_word;     /* [1]   EP_DEVERR_* bits */
 } ep_handle;
 
-/* Version of this ABI (EP_ABI_VERSION). */
+/* Version of this ABI (EP_ABI_VERSION).  The pages have no counterpart:
+ * this and the two calls below are the C ABI's own error reporting. */
 EP_API int32_t ep_abi_version(void);
 
 /* Human-readable name of a status code; never NULL. */
@@ -113,18 +114,24 @@ EP_API const char* ep_last_error(void);
 
 /* Worst-case receive rows T*k + E*(a-1): the size to give recv_x, recv_src,
  * recv_topk_idx / weights and y so that any routing fits.  -1 on bad
- * arguments or int32 overflow. */
+ * arguments or int32 overflow.  Stands for the buffer sizing of the DeepEP
+ * V2 README, "Interfaces and examples" (get_buffer_size_hint from
+ * num_max_tokens_per_rank, hidden and top-k), here for caller-owned
+ * receive tensors instead of a library-owned communication buffer. */
 EP_API int32_t ep_max_recv_rows(int32_t num_tokens, int32_t num_topk, int32_t num_experts,
                                 int32_t expert_alignment);
 
 /* Bytes of the device block that ep_handle_init carves up (0 on bad
- * arguments).  Limits: T >= 0, 1 <= k <= 32, 1 <= E <= 1024, S >= 1 and
+ * arguments): the storage of the handle (EPHandle, DeepEP V2 README,
+ * "Interfaces and examples") that dispatch returns and combine reuses.  Limits: T >= 0, 1 <= k <= 32, 1 <= E <= 1024, S >= 1 and
  * S divides E, a >= 1, max_recv_rows >= ep_max_recv_rows(T, k, E, a). */
 EP_API size_t ep_handle_bytes(int32_t num_tokens, int32_t num_topk, int32_t num_experts,
                               int32_t num_segments, int32_t expert_alignment,
                               int32_t max_recv_rows);
 
-/* Fills *handle with pointers into `device_block` (at least
+/* The handle (EPHandle, DeepEP V2 README, "Interfaces and examples") as a
+ * plain struct of device pointers.  Fills *handle with pointers into
+ * `device_block` (at least
  * ep_handle_bytes() bytes, 256-byte aligned, owned by the caller and kept
  * alive as long as the handle is used) and zeroes nothing: the layout
  * writes every field before use.  Host only; launches nothing. */
@@ -173,8 +180,10 @@ EP_API ep_status ep_get_layout(ep_handle* handle, const void* topk_idx, int32_t 
  * (for E = 256 experts about a million slots fit).  Allocates and frees
  * nothing.  The first call on each device looks up the array's device
  * address (cudaGetSymbolAddress) with that device current, so make that
- * first call before any stream capture.  All calls share the array: calls
- * that overlap on the GPU race on it. */
+ * first call before any stream capture.  That address is kept until the
+ * process exits: a cudaDeviceReset of the device after the first call is
+ * not supported (the kept address would be stale).  All calls share the
+ * array: calls that overlap on the GPU race on it. */
 EP_API ep_status ep_get_layout_static(ep_handle* handle, const void* topk_idx, int32_t idx_is_int64,
                                       const float* topk_weights, int32_t* recv_topk_idx,
                                       float* recv_topk_weights, ep_stream_t stream);
@@ -268,12 +277,17 @@ EP_API ep_status ep_combine_backward(const ep_handle* handle, const void* grad_o
                                      int32_t hidden, const float* topk_weights, void* grad_y,
                                      float* grad_weights, ep_stream_t stream);
 
-/* Copies R = offsets[E] to *total_rows on the host.  Synchronises `stream`. */
+/* Copies R = offsets[E] to *total_rows on the host.  Synchronises `stream`.
+ * This is the host read that the README's decode example ("Interfaces and
+ * examples": a cached handle avoids a redundant CPU sync) keeps off the hot
+ * path; every other call leaves R on the device. */
 EP_API ep_status ep_read_total_rows(const ep_handle* handle, int32_t* total_rows,
                                     ep_stream_t stream);
 
 /* Reads the device error word into *bits (may be NULL) and clears it.
- * Synchronises `stream`.  Returns EP_ERR_DEVICE if any bit was set. */
+ * Synchronises `stream`.  Returns EP_ERR_DEVICE if any bit was set.  The
+ * pages have no counterpart (their kernels assert); this is the sync the
+ * README's decode example avoids, taken only when the caller asks. */
 EP_API ep_status ep_check_error(const ep_handle* handle, uint32_t* bits, ep_stream_t stream);
 
 #ifdef __cplusplus

@@ -54,5 +54,31 @@ def test_combine_traffic_is_read_only_for_the_profiled_source_and_workload():
     assert bench.combine_traffic("mid", 8192) is None
 
 
+def test_combine_traffic_comes_from_the_json_record(tmp_path, monkeypatch):
+    # the record is machine-readable: read + write bytes, keyed by the kernel
+    # source's sha256 prefix, the workload and T
+    import hashlib
+    import json
+    import os
+    src = tmp_path / "combine_ep_get_06_b200" / "csrc"
+    src.mkdir(parents=True)
+    (src / "combine.cu").write_bytes(b"// some kernel\n")
+    sha = hashlib.sha256(b"// some kernel\n").hexdigest()[:16]
+    (tmp_path / "profiles").mkdir()
+    rec = {"combine_kernel": {"workload": "v3", "T": 8192, "source_sha16": sha,
+                              "dram_read_bytes": 940, "dram_write_bytes": 65}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.combine_traffic("v3", 8192) == 1005
+    (src / "combine.cu").write_bytes(b"// changed\n")           # kernel changed since the capture
+    assert bench.combine_traffic("v3", 8192) is None
+    assert os.path.exists(tmp_path / "profiles" / "traffic.json")
+
+
+def test_line_labels():
+    # the arithmetic the path computes in, not a precision claim
+    assert "e4m3" in bench.DTYPE and "f32" in bench.DTYPE
+
+
 def test_weak_scaling_sums_bytes_over_ranks():
     assert np.isclose(bench.weak_scaling_gbs(1_000_000_000, 4, 2.0), 4 * 1.0 / 2e-3)

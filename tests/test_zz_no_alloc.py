@@ -4,7 +4,9 @@ every device allocation, or plain C code with no device allocator), so
 cannot pass ep_get_layout a workspace.  Its scratch lives in a fixed array
 inside the library.  Through the C ABI, it must give exactly what
 ep_get_layout gives with a caller-owned workspace, call after call, and
-must refuse a layout too large for that array.
+must refuse a layout too large for that array.  Its results are also
+compared with the CPU oracle's layout directly, not only through the
+workspace entry.
 
 This file is named so that pytest collects it last."""
 
@@ -14,6 +16,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import workloads as W
 from combine_ep_get_06_b200 import ep as B
 
@@ -37,8 +40,10 @@ def test_static_scratch_layout_equals_workspace_layout_on_consecutive_calls():
         pytest.skip("no CUDA device")
     L = B.lib()
     stream = torch.cuda.current_stream().cuda_stream
-    # many chunks, so the per-chunk histograms really pass through the scratch
-    for name, idx_dtype in (("v3", torch.int64), ("mid", torch.int32)):
+    # v3 and mid have many chunks, so the per-chunk histograms really pass
+    # through the scratch; decode (T*k = 1024) is one chunk, which never
+    # touches it but still goes through the size check and the address
+    for name, idx_dtype in (("v3", torch.int64), ("mid", torch.int32), ("decode", torch.int64)):
         w = W.WORKLOADS[name]
         ref_h = B.EPHandle(w.T, w.k, w.E, w.S, w.align)
         new_h = B.EPHandle(w.T, w.k, w.E, w.S, w.align)
@@ -61,6 +66,15 @@ def test_static_scratch_layout_equals_workspace_layout_on_consecutive_calls():
             for key in ref:
                 np.testing.assert_array_equal(new[key], ref[key], err_msg=f"{name} seed {seed}: {key}")
             assert new_h.check_error() == 0
+            lay = oracle.layout(inp["topk_idx"], w.E, w.S, w.align, inp["topk_weights"])
+            R = int(lay["R"])
+            np.testing.assert_array_equal(new["counts"], lay["counts"])
+            np.testing.assert_array_equal(new["offsets"], lay["offsets"])
+            np.testing.assert_array_equal(new["seg_tokens"], lay["seg_tokens"])
+            np.testing.assert_array_equal(new["slot_map"], lay["slot_map"])
+            np.testing.assert_array_equal(new["recv_src"], lay["recv_src"][:R])
+            np.testing.assert_array_equal(new["recv_topk_idx"], lay["recv_topk_idx"][:R])
+            np.testing.assert_array_equal(new["recv_topk_weights"], lay["recv_topk_weights"][:R].view(np.uint32))
 
 
 def test_static_scratch_layout_refuses_layouts_larger_than_its_array():
