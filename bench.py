@@ -221,6 +221,7 @@ def time_back_to_back(fn, n: int, stream) -> float:
     for _ in range(3):
         fn()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(1_000_000)   # let the host queue the calls before the start event
     a.record(stream)
     for _ in range(n):
         fn()
@@ -359,8 +360,10 @@ def run_ours(args, rank, world, dev):
     nbytes = step_bytes(w, T, V, P, R)
     handle.check_error()
 
+    # The timed region: K steps with nothing between the calls, so each
+    # kernel may launch while the one before it drains (programmatic
+    # dependent launch); an event recorded between two kernels would stop it.
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(nvsmi_device_id(dev))
     if world > 1:
@@ -368,18 +371,30 @@ def run_ours(args, rank, world, dev):
     torch.cuda.synchronize(dev)
     sampler.start()
     time.sleep(0.3)
+    # Hold the stream for ~0.5 ms (torch's bounded sleep kernel, before the
+    # start event) so that the host has queued the first steps when timing
+    # starts: the timed region then holds device time only.
+    torch.cuda._sleep(1_000_000)
     start.record(stream)
-    for i in range(K):
-        e = ev[i]
-        e[0].record(stream); layout_dispatch()
-        e[1].record(stream); combine()
-        e[2].record(stream)
+    for _ in range(K):
+        layout_dispatch()
+        combine()
     end.record(stream)
     torch.cuda.synchronize(dev)
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
     total_ms = start.elapsed_time(end)
+
+    # Per-kernel breakdown after the timed region: the same step with an
+    # event between the calls (slightly slower for it).
+    K3 = max(5, min(50, K))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K3)]
+    for e in ev:
+        e[0].record(stream); layout_dispatch()
+        e[1].record(stream); combine()
+        e[2].record(stream)
+    torch.cuda.synchronize(dev)
     ld_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     com_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
     handle.check_error()
@@ -402,9 +417,8 @@ def run_ours(args, rank, world, dev):
         e[3].record(stream)
     torch.cuda.synchronize(dev)
     lay_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev2)
-    two_dis_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev2)
+    dis_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev2)
     two_step_ms = statistics.mean(e[0].elapsed_time(e[3]) for e in ev2)
-    dis_ms = time_back_to_back(dispatch, K2, stream)
     handle.check_error()
 
     def rate(nb, ms):
@@ -420,11 +434,13 @@ def run_ours(args, rank, world, dev):
         "gpu_launches": K * (layout_launches(T, k) + 2),
         "step": "ep_layout_dispatch (layout + FP8 dispatch, one call) -> ep_combine",
         "layout_dispatch": {**rate(nbytes["layout"] + nbytes["dispatch"], ld_ms),
-                            "note": "in the timed step: layout kernels and the dispatch kernel of one call"},
+                            "note": "layout kernels and the dispatch kernel of one call, inside the step (events "
+                                    "between the calls, after the timed region)"},
         "combine": rate(nbytes["combine"], com_ms),
         "dispatch": {**rate(nbytes["dispatch"], dis_ms), "valid_rows": V, "padding_rows": P,
-                     "note": "the dispatch kernel alone, back to back after the timed step"},
-        "two_call": {"layout_us": round(lay_ms * 1e3, 2), "dispatch_us": round(two_dis_ms * 1e3, 2),
+                     "note": "the dispatch kernel between the layout and the combine of a two-call step "
+                             "(ep_get_layout, ep_dispatch, ep_combine), after the timed step"},
+        "two_call": {"layout_us": round(lay_ms * 1e3, 2), "dispatch_us": round(dis_ms * 1e3, 2),
                      "step_us": round(two_step_ms * 1e3, 2),
                      "note": "ep_get_layout, ep_dispatch, ep_combine as separate calls"},
         "clocks": clocks,
@@ -459,6 +475,13 @@ def run_ours(args, rank, world, dev):
         c8_bytes = V * (H + (H // 128) * 4) + T * k * 8 + T * H * 2
         res["combine_fp8"] = rate(c8_bytes, time_back_to_back(c8, n_x, stream))
 
+    # dispatch and combine on a bounded number of SMs (the pages' #SMs column), same workload
+    res["sm_budget"] = {"note": "dispatch and combine kernels alone, each CTA filling one SM, at most n SMs"}
+    for n_sms in (24, 64):
+        with ep.sm_budget(n_sms):
+            res["sm_budget"][str(n_sms)] = {"dispatch": rate(nbytes["dispatch"], time_back_to_back(dispatch, n_x, stream)),
+                                            "combine": rate(nbytes["combine"], time_back_to_back(combine, n_x, stream))}
+
     # the backward of the weighted combine (training), same workload
     gy = torch.empty(rows, H, dtype=torch.bfloat16, device=dev)
     gw = torch.empty(T, k, dtype=torch.float32, device=dev)
@@ -484,8 +507,8 @@ def run_ours(args, rank, world, dev):
 
 def run_workload_lines(args, dev, name: str, peak: float) -> dict:
     """Dispatch and combine GB/s on another workload (its own seeded inputs):
-    the step (one-call layout + dispatch, then combine) per call, and the
-    dispatch and combine kernels alone, back to back."""
+    the step (one-call layout + dispatch, then combine), and the dispatch and
+    combine kernels timed inside a two-call step (layout, dispatch, combine)."""
     import torch
 
     import combine_ep_get_06_b200 as ep
@@ -510,12 +533,22 @@ def run_workload_lines(args, dev, name: str, peak: float) -> dict:
     stream = torch.cuda.current_stream(dev)
     one = lambda: ep.dispatch(x, idx, wts, w.E, expert_alignment=w.align, num_segments=w.S, handle=handle,
                               use_fp8=fp8, recv_x=recv_x, recv_scales=recv_s)
+    lay = lambda: ep.get_layout(idx, w.E, num_segments=w.S, expert_alignment=w.align, topk_weights=wts,
+                                handle=handle)
     dis = lambda: ep.dispatch_with_handle(x, handle, use_fp8=fp8, recv_x=recv_x, recv_scales=recv_s)
     com = lambda: ep.combine(y, handle, wts, out=out)
     n = max(5, min(50, args.steps))
     step_ms = time_back_to_back(lambda: (one(), com()), n, stream)
-    dis_ms = time_back_to_back(dis, n, stream)
-    com_ms = time_back_to_back(com, n, stream)
+    # the kernels inside a two-call step, each between its neighbours (as in the timed V3 step)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
+    for e in ev:
+        e[0].record(stream); lay()
+        e[1].record(stream); dis()
+        e[2].record(stream); com()
+        e[3].record(stream)
+    torch.cuda.synchronize(dev)
+    dis_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    com_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
     handle.check_error()
     V = int(handle.counts.sum())
     P = int(handle.num_pad_rows[0])

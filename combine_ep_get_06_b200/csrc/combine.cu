@@ -2,10 +2,12 @@
 // combine_forward, and dispatch_backward when unweighted).
 //
 // out[t] = bf16( sum_j w[t,j] * y[slot_map[t*k+j]] ) over the valid slots,
-// fp32 FMA from +0 in ascending j, one bf16 rounding at the end.  A CTA
-// works on one unit = blockDim 16-byte column items (8 bf16) of one token:
-// each thread issues its (up to 8 per group) row loads before the FMAs, so
-// a thread keeps k 16-byte loads in flight.  Launched with programmatic
+// fp32 FMA from +0 in ascending j, one bf16 rounding at the end.  A unit is
+// `ut` 16-byte column items (8 bf16) of one token, one item per thread: each
+// thread issues its (up to 8 per group) row loads before the FMAs, so a
+// thread keeps k 16-byte loads in flight.  A CTA is blockDim / ut groups of
+// ut threads, each working through units on its own (one group normally;
+// under an SM budget enough groups to fill an SM with one CTA).  Launched with programmatic
 // dependent launch: the CTAs start while the previous grid finishes and
 // wait for it before reading anything; each lets the next grid start
 // launching once its own work is issued.
@@ -15,11 +17,19 @@
 namespace ep {
 namespace {
 
-constexpr int kMaxThreads = 256;
+constexpr int kMaxThreads = 256;  // threads of a unit at most
 
-template <int G>  // groups of 8 slots: k <= 8 * G
-__global__ void __launch_bounds__(kMaxThreads) combine_kernel(CombineArgs a, int ipr, int upr) {
+// Threads of a CTA under an SM budget, for k <= 8*G: as many as fit an SM
+// without spilling the k row values a thread holds.
+template <int G>
+constexpr int budget_threads() {
+    return G == 1 ? 1024 : 256;
+}
+
+template <int G, int kMaxT>  // groups of 8 slots: k <= 8 * G; at most kMaxT threads
+__global__ void __launch_bounds__(kMaxT) combine_kernel(CombineArgs a, int ipr, int upr, int ut) {
     const int tid = threadIdx.x;
+    const int nsub = blockDim.x / ut, sub = tid / ut, lt = tid - sub * ut;
     const int T = a.T, k = a.k, H = a.H;
     const char* const y = (const char*)a.y;
     const size_t row_bytes = (size_t)H * 2;
@@ -35,9 +45,10 @@ __global__ void __launch_bounds__(kMaxThreads) combine_kernel(CombineArgs a, int
     }
 
     const int64_t n_units = (int64_t)T * upr;
-    for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
+    const int64_t u0 = sub < nsub ? (int64_t)blockIdx.x * nsub + sub : n_units;
+    for (int64_t u = u0; u < n_units; u += (int64_t)gridDim.x * nsub) {
         const int t = (int)(u / upr);
-        const int c = (int)(u - (int64_t)t * upr) * blockDim.x + tid;
+        const int c = (int)(u - (int64_t)t * upr) * ut + lt;
         if (c >= ipr) continue;
 
         int rows[8 * G];
@@ -97,18 +108,17 @@ int unit_threads(int ipr) {
     return ipr < kMaxThreads ? ((ipr + 31) / 32) * 32 : kMaxThreads;
 }
 
-template <int G>
-cudaError_t launch_t(const CombineArgs& a, cudaStream_t stream) {
-    const int ipr = a.H / 8;
-    const int bd = unit_threads(ipr);
-    const int upr = (ipr + bd - 1) / bd;
+template <int G, int kMaxT>
+cudaError_t launch_bd(const CombineArgs& a, int ipr, int ut, int bd, int max_ctas, cudaStream_t stream) {
+    const int upr = (ipr + ut - 1) / ut;
+    auto kernel = combine_kernel<G, kMaxT>;
     int per_sm = 0;
-    cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_kernel<G>, bd, 0);
+    cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, bd, 0);
     if (err != cudaSuccess) return err;
     if (per_sm < 1) per_sm = 1;
     // Persistent grid, no larger than the work.
-    const int64_t cap = (int64_t)device_sm_count() * per_sm;
-    int64_t want = (int64_t)a.T * upr;
+    const int64_t cap = max_ctas > 0 ? max_ctas : (int64_t)device_sm_count() * per_sm;
+    int64_t want = ((int64_t)a.T * upr + bd / ut - 1) / (bd / ut);
     if (a.out_weights != nullptr) {
         const int64_t gather = ((int64_t)a.T * a.k + bd - 1) / bd;
         if (gather > want) want = gather;
@@ -123,7 +133,22 @@ cudaError_t launch_t(const CombineArgs& a, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, combine_kernel<G>, a, ipr, upr);
+    debug_launch("combine_kernel", G, cfg);
+    return cudaLaunchKernelEx(&cfg, kernel, a, ipr, upr, ut);
+}
+
+// One unit group per CTA and as many CTAs as fit; under an SM budget of n,
+// n CTAs of as many unit groups as fit budget_threads<G>(), one CTA to an SM.
+template <int G>
+cudaError_t launch_t(const CombineArgs& a, cudaStream_t stream) {
+    const int ipr = a.H / 8;
+    const int ut = unit_threads(ipr);
+    const int budget = sm_budget();
+    if (budget > 0) {
+        constexpr int kT = budget_threads<G>();
+        return launch_bd<G, kT>(a, ipr, ut, (kT / ut) * ut, budget, stream);
+    }
+    return launch_bd<G, kMaxThreads>(a, ipr, ut, ut, 0, stream);
 }
 
 }  // namespace

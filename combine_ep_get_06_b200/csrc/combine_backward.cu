@@ -145,6 +145,7 @@ cudaError_t launch_t(const CombineBackwardArgs& a, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    debug_launch("combine_backward_kernel", G, cfg);
     return cudaLaunchKernelEx(&cfg, combine_backward_kernel<G>, a, ipr);
 }
 

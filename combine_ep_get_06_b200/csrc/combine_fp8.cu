@@ -128,6 +128,7 @@ cudaError_t launch_t(const CombineFp8Args& a, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    debug_launch("combine_fp8_kernel", G, cfg);
     return cudaLaunchKernelEx(&cfg, combine_fp8_kernel<G>, a, ipr, upr);
 }
 

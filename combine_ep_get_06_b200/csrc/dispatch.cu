@@ -1,196 +1,256 @@
 // MoE dispatch on one device (DeepEP V2 README, "Interfaces and examples",
 // dispatch_forward; FP8 dispatching as in its section "Performance").
 //
-// Token-major: each token row is read from HBM once and, in the FP8 mode,
-// quantised once, into a shared-memory row buffer; the TMA engine then
-// copies that buffer to each of the token's k receive rows with bulk
-// shared->global copies (cp.async.bulk, never multicast), so the SMs issue
-// a handful of copy instructions per row instead of k stores per 16 bytes.
-// Two row buffers alternate, so filling row i+1 overlaps the copies of row
-// i, and the loads of a CTA's next row are issued as soon as the current
-// row is in shared memory, so they are in flight across the barrier and
-// the copy issue.  Padding rows are written by bulk copies of a zeroed
-// buffer, one row per lane of warp 0.
+// Warp-granular: the unit of work is one warp's, and warps never wait on
+// one another (no CTA barrier after the start).  A unit is either
+//   - a token slice: 1024 consecutive elements of one token row.  The warp
+//     loads them (16 bytes a lane per load, a warp load covers 512
+//     contiguous bytes), converts them (FP8: amax over the 1x128 block, 16
+//     lanes, by xor shuffles; scale and inverse by IEEE division; e4m3
+//     conversion) into a per-warp shared-memory stage, and lanes j < k
+//     copy the stage to the slice of receive row slot_map[t*k+j] with TMA
+//     bulk copies (cp.async.bulk shared->global, never multicast); or
+//   - a padding row: lanes copy a zeroed buffer over the row's slices.
+// Units are numbered token-major (t, slice), then padding rows, and dealt
+// to the warps grid-stride, so every warp gets the same mix of small units
+// and the grid has no long tail.  Each warp keeps its next unit's loads
+// and routing in flight while it converts and copies the current one, and
+// cycles kStages stages: a stage is refilled only once the copies issued
+// from it kStages units ago have read it.
 //
-// A CTA walks rows grid-stride: token rows [0, T), then padding batches of
-// 32 rows.  Launched with programmatic dependent launch: a CTA waits for
-// the previous grid before reading what it may have written (directly after
-// the layout, only the routing), and lets the next grid start launching
-// once it has issued all its copies.
-#include "dispatch_device.cuh"
+// Launched with programmatic dependent launch: the first unit's x loads
+// may be issued before waiting for the previous grid (only directly after
+// the layout, which leaves x untouched), everything the layout writes is
+// read after the wait, and the next grid may start launching once all
+// copies are issued.
+#include "dispatch_warp.cuh"
 
 namespace ep {
 namespace {
 
-using namespace dispatch_dev;
+using namespace warp_units;
 
-constexpr int kThreads = 256;
-constexpr int kPre = 2;  // 32-item slices per warp whose loads are prefetched
-constexpr int kBuf = 2;  // row buffers: a buffer is refilled once the copies from kBuf rows ago have read it
+constexpr int kWarps = 8;         // warps per CTA; two CTAs to an SM
+constexpr int kBudgetWarps = 24;  // warps per CTA under an SM budget: one CTA fills an SM
+constexpr int kStages = 4;
+constexpr int kPrefetchUnits = 3;  // units after the first whose x is brought into L2 during the layout
 
-// smem: [kBuf][row_bytes] row buffers | [kBuf][scale_pad] scale buffers |
-//       [row_bytes] zeros | [scale_pad] zeros | [kBuf][kMaxTopk] int rows
-__host__ __device__ inline size_t smem_bytes(const Geometry& g) {
-    return (size_t)(kBuf + 1) * g.row_bytes + (size_t)(kBuf + 1) * g.scale_pad + kBuf * kMaxTopk * sizeof(int);
+__host__ __device__ inline size_t smem_bytes(const SliceGeo& g, int warps) {
+    return (size_t)g.stage_bytes * (1 + warps * kStages);  // zero buffer + the warps' stages
 }
 
-// Stores the scale of block b of receive row `row` (f32 row- or MN-major,
-// or an e4m3 byte for NVFP4), taken from the row's scale buffer sb.
-// MN-major scales are stored with an L2 evict-last policy: each token's
-// scales land in B different columns, 4 bytes per 32-byte sector, and the
-// whole array fits in L2, so its sectors fill up there before write-back
-// (measured: 158 -> 134 us at the V3 shape).  A hint on the row copies
-// measured slower and is not used.
+// The routing of unit u, read from the handle (which the previous grid,
+// the layout, may have written).
 template <int kMode>
-__device__ __forceinline__ void store_scale(const DispatchArgs& a, int row, int b, const float* sb, bool zero,
-                                            uint64_t keep) {
+__device__ __forceinline__ Meta load_meta(const DispatchArgs& a, const SliceGeo& g, int64_t u,
+                                          int64_t n_tok_units, int64_t n_units, int lane) {
+    Meta m;
+    m.row = -1;
+    m.xs = 0.0f;
+    if (u >= n_units) return m;
+    if (u >= n_tok_units) {
+        m.row = ld_cg(a.pad_rows + (u - n_tok_units));
+        return m;
+    }
+    const int t = (int)(u / g.ns), s = (int)(u - (int64_t)t * g.ns);
+    if (lane < a.k) m.row = ld_cg(a.slot_map + (size_t)t * a.k + lane);
+    if (kMode == EP_X_FP8) {
+        const int nb = min(kSliceElems, a.H - s * kSliceElems) / 128;
+        if (lane < nb) m.xs = ld_cg(a.x_scales + (size_t)t * (a.H / 128) + s * (kSliceElems / 128) + lane);
+    }
+    return m;
+}
+
+// Stores scale b of receive row `row`: f32 row-major or MN-major (the
+// latter under an L2 evict-last policy: each token's scales land in B
+// different columns, 4 bytes per 32-byte sector, and the whole array fits
+// in L2, so its sectors fill up there before write-back), or an e4m3 byte
+// for NVFP4.
+template <int kMode>
+__device__ __forceinline__ void store_scale(const DispatchArgs& a, int row, int b, const unsigned char* sst,
+                                            int bi, uint64_t keep) {
     if (kMode == EP_X_BF16_TO_NVFP4) {
-        reinterpret_cast<unsigned char*>(a.recv_scales)[(size_t)row * (a.H / 16) + b] =
-            zero ? 0 : reinterpret_cast<const unsigned char*>(sb)[b];
-    } else if (a.scales_ld > 0) {
-        st_f32_hint(reinterpret_cast<float*>(a.recv_scales) + (size_t)b * a.scales_ld + row, zero ? 0.0f : sb[b],
-                    keep);
+        reinterpret_cast<unsigned char*>(a.recv_scales)[(size_t)row * (a.H / 16) + b] = sst ? sst[bi] : 0;
     } else {
-        reinterpret_cast<float*>(a.recv_scales)[(size_t)row * (a.H / 128) + b] = zero ? 0.0f : sb[b];
+        const float v = sst ? reinterpret_cast<const float*>(sst)[bi] : 0.0f;
+        if (a.scales_ld > 0)
+            st_f32_hint(reinterpret_cast<float*>(a.recv_scales) + (size_t)b * a.scales_ld + row, v, keep);
+        else
+            reinterpret_cast<float*>(a.recv_scales)[(size_t)row * (a.H / 128) + b] = v;
     }
 }
 
-
+// Whether the scales of a slice of ne elements go out as one bulk copy:
+// scale rows a multiple of 16 bytes in a 16-byte aligned array (the host
+// sets bulk_scales; never for MN-major scales), and the slice's scale
+// bytes a multiple of 16.
 template <int kMode>
-__device__ __forceinline__ void prefetch(const DispatchArgs& a, int t, int ipr, Item (&p)[kPre]) {
+__device__ __forceinline__ bool bulk_scales_ok(const DispatchArgs& a, int ne) {
+    return a.bulk_scales && (ne / Mode<kMode>::kScaleBlock * Mode<kMode>::kScaleBytes) % 16 == 0;
+}
+
+// Zeroes the zero buffer at the start of `smem` (a barrier follows in the caller).
+template <int kW>
+__device__ __forceinline__ void zero_buffer(unsigned char* zeros, int bytes) {
+    for (int i = threadIdx.x; i < bytes / 16; i += 32 * kW) reinterpret_cast<uint4*>(zeros)[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+}
+
+// The unit loop of one warp, from unit u on (its x loads already in nxt),
+// then the end of the grid's work.  `smem` holds the zero buffer and then
+// kStages stages per warp.
+template <int kMode, int kW>
+__device__ __forceinline__ void run_units(const DispatchArgs& a, const SliceGeo& g, unsigned char* smem,
+                                          int64_t u, Loads<kMode> nxt, int64_t n_pad) {
+    using M = Mode<kMode>;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int i = 0; i < kPre; ++i) {
-        const int c = warp * 32 + i * kThreads + lane;
-        p[i] = load_item<kMode>(a, t, c, t < a.T && c < ipr);
-    }
-}
-
-template <int kMode>
-__global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchArgs a) {
-    constexpr bool kFp8Out = kMode != EP_X_BF16;
-    extern __shared__ __align__(128) unsigned char smem[];
-    const Geometry geo = geometry(kMode, a.H);
-    unsigned char* rowbuf = smem;                                  // [kBuf][row_bytes]
-    unsigned char* sclbuf = smem + kBuf * geo.row_bytes;           // [kBuf][scale_pad]
-    unsigned char* zeros = sclbuf + kBuf * geo.scale_pad;          // [row_bytes + scale_pad]
-    int* rows_s = (int*)(zeros + geo.row_bytes + geo.scale_pad);   // [kBuf][kMaxTopk]
-
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int T = a.T, k = a.k;
-    const int B = kMode == EP_X_BF16_TO_NVFP4 ? a.H / 16 : a.H / 128;  // scales per row
+    unsigned char* const zeros = smem;  // [stage_bytes] of zeros
+    unsigned char* const stages = smem + (size_t)g.stage_bytes * (1 + warp * kStages);
     char* const recv = (char*)a.recv_x;
     char* const rscl = (char*)a.recv_scales;
-
-    for (int i = tid; i < (geo.row_bytes + geo.scale_pad) / 16; i += kThreads)
-        reinterpret_cast<uint4*>(zeros)[i] = make_uint4(0, 0, 0, 0);
-    fence_proxy_async_smem();
+    const int k = a.k;
     const uint64_t keep = a.scales_ld > 0 ? l2_evict_last_policy() : 0;
+    const int64_t n_tok_units = (int64_t)a.T * g.ns;
+    const int64_t stride = (int64_t)gridDim.x * kW;
+    const int64_t n_units = n_tok_units + n_pad;
+    Meta nmeta = load_meta<kMode>(a, g, u, n_tok_units, n_units, lane);
 
-    // Right after the layout x is already complete (every layout kernel waits
-    // for the grid before it before letting this one launch), so the first
-    // row's loads can fly while the layout finishes.  Everything the layout
-    // writes is read only after the wait.
-    Item next[kPre];
-    if (a.x_ready) prefetch<kMode>(a, blockIdx.x, geo.ipr, next);
-    pdl_wait();
-    if (!a.x_ready) prefetch<kMode>(a, blockIdx.x, geo.ipr, next);
-    const int n_pad = ld_cg(a.num_pad_rows);
-    const int n_pad_batches = (n_pad + 31) / 32;
-    __syncthreads();
+    int it = 0;  // token units of this warp (selects the stage)
+    for (; u < n_units; u += stride) {
+        const Loads<kMode> cur = nxt;
+        const Meta m = nmeta;
+        {
+            const int64_t un = u + stride;
+            nxt = load_x<kMode>(a, g, un, n_tok_units, lane);
+            nmeta = load_meta<kMode>(a, g, un, n_tok_units, n_units, lane);
+        }
 
-    int it = 0;  // token rows handled by this CTA (selects the buffer)
-    for (int r = blockIdx.x; r < T + n_pad_batches; r += gridDim.x) {
-        if (r >= T) {
-            // 32 padding rows: one bulk copy of zeros per row (lanes of warp 0).
-            const int p = (r - T) * 32 + lane;
-            if (warp == 0 && p < n_pad) {
-                const int row = ld_cg(a.pad_rows + p);
-                if (row >= 0 && row < a.max_rows) {
-                    bulk_s2g(recv + (size_t)row * geo.row_bytes, zeros, geo.row_bytes);
-                    if (a.bulk_scales)
-                        bulk_s2g(rscl + (size_t)row * geo.scale_bytes, zeros + geo.row_bytes, geo.scale_bytes);
-                    bulk_commit();
-                    if (kFp8Out && !a.bulk_scales)
-                        for (int b = 0; b < B; ++b) store_scale<kMode>(a, row, b, nullptr, true, keep);
+        if (u >= n_tok_units) {
+            // A padding row: zero data and scales.
+            const int row = m.row;
+            if (row < 0 || row >= a.max_rows) {
+                if (row >= a.max_rows && lane == 0) atomicOr(a.error_word, EP_DEVERR_CAPACITY);
+                continue;
+            }
+            if (!EP_CHECK(u - n_tok_units < n_pad, a.error_word)) continue;
+            for (int s = lane; s < g.ns; s += 32) {
+                const int ne = min(kSliceElems, a.H - s * kSliceElems);
+                bulk_s2g(recv + (size_t)row * g.row_bytes + (size_t)s * g.out_bytes, zeros,
+                         ne * g.out_bytes / kSliceElems);
+                if (M::kScales && bulk_scales_ok<kMode>(a, ne))
+                    bulk_s2g(rscl + (size_t)row * g.srow_bytes + (size_t)s * g.sout_bytes, zeros,
+                             ne / M::kScaleBlock * M::kScaleBytes);
+            }
+            bulk_commit();
+            if (M::kScales) {
+                constexpr int kPerSlice = kSliceElems / M::kScaleBlock;
+                const int B = a.H / M::kScaleBlock;
+                for (int b = lane; b < B; b += 32) {
+                    const int s = b / kPerSlice;
+                    if (!bulk_scales_ok<kMode>(a, min(kSliceElems, a.H - s * kSliceElems)))
+                        store_scale<kMode>(a, row, b, nullptr, 0, keep);
                 }
             }
             continue;
         }
 
-        const int t = r;
-        const int buf = it % kBuf;
+        // A token slice.
+        const int t = (int)(u / g.ns), s = (int)(u - (int64_t)t * g.ns);
+        const int ne = min(kSliceElems, a.H - s * kSliceElems);
+        unsigned char* const st = stages + (size_t)(it % kStages) * g.stage_bytes;
+        unsigned char* const sst = st + g.out_bytes;
         ++it;
-        unsigned char* rb = rowbuf + buf * geo.row_bytes;
-        float* sb = reinterpret_cast<float*>(sclbuf + buf * geo.scale_pad);
-        int* rows = rows_s + buf * kMaxTopk;
-
-        // The copies issued kBuf rows ago from this buffer must have read it
-        // (each lane below k commits one bulk group per token row).
-        if (warp == 0) bulk_wait_read<kBuf - 1>();
-        __syncthreads();
-
-        if (tid < k) rows[tid] = ld_cg(a.slot_map + (size_t)t * k + tid);
-
-        // Fill the row buffer: the prefetched slices, then any further ones.
-#pragma unroll
-        for (int i = 0; i < kPre; ++i) {
-            const int c0 = warp * 32 + i * kThreads;
-            if (c0 < geo.ipr) fill_item<kMode>(a, t, c0 + lane, c0 + lane < geo.ipr, next[i], rb, sb);
-        }
-        for (int c0 = warp * 32 + kPre * kThreads; c0 < geo.ipr; c0 += kThreads) {
-            const int c = c0 + lane;
-            fill_item<kMode>(a, t, c, c < geo.ipr, load_item<kMode>(a, t, c, c < geo.ipr), rb, sb);
-        }
-        // This CTA's next token row: its loads fly across the barrier and copy issue.
-        prefetch<kMode>(a, r + gridDim.x, geo.ipr, next);
+        // The copies issued from this stage kStages units ago must have read it.
+        if (lane < k) bulk_wait_read<kStages - 1>();
+        __syncwarp();
+        fill_stage<kMode>(cur, m, ne, lane, st, sst);
         fence_proxy_async_smem();
-        __syncthreads();
+        __syncwarp();
 
-        if (warp == 0 && lane < k) {
-            const int row = rows[lane];
-            if (row >= 0 && row < a.max_rows) {
-                bulk_s2g(recv + (size_t)row * geo.row_bytes, rb, geo.row_bytes);
-                if (a.bulk_scales) bulk_s2g(rscl + (size_t)row * geo.scale_bytes, sb, geo.scale_bytes);
+        const int sb = M::kScales ? ne / M::kScaleBlock * M::kScaleBytes : 0;
+        const bool bulk_scl = M::kScales && bulk_scales_ok<kMode>(a, ne);
+        if (lane < k) {
+            const int row = m.row;
+            const int db = ne * g.out_bytes / kSliceElems;
+            if (row >= 0 && row < a.max_rows &&
+                EP_CHECK(t < a.T && (size_t)s * g.out_bytes + db <= (size_t)g.row_bytes &&
+                             (size_t)s * g.sout_bytes + sb <= (size_t)g.srow_bytes,
+                         a.error_word)) {
+                bulk_s2g(recv + (size_t)row * g.row_bytes + (size_t)s * g.out_bytes, st, db);
+                if (bulk_scl) bulk_s2g(rscl + (size_t)row * g.srow_bytes + (size_t)s * g.sout_bytes, sst, sb);
             } else if (row >= a.max_rows) {
                 atomicOr(a.error_word, EP_DEVERR_CAPACITY);
             }
             bulk_commit();
         }
-        if (kFp8Out && !a.bulk_scales) {
-            // MN-major scales, or rows not a multiple of 16 bytes: plain stores.
-            for (int i = tid; i < k * B; i += kThreads) {
-                const int row = rows[i / B];
-                if (row >= 0 && row < a.max_rows) store_scale<kMode>(a, row, i % B, sb, false, keep);
+        if (M::kScales && !bulk_scl) {
+            // MN-major scales, or scale rows that are not a multiple of 16 bytes: plain stores.
+            const int nb = ne / M::kScaleBlock, b0 = s * (kSliceElems / M::kScaleBlock);
+            for (int j = 0; j < k; ++j) {
+                const int row = __shfl_sync(0xffffffffu, m.row, j);
+                if (row < 0 || row >= a.max_rows) continue;
+                for (int b = lane; b < nb; b += 32) store_scale<kMode>(a, row, b0 + b, sst, b, keep);
             }
         }
     }
     // Let the next grid start launching while the copies drain.
     pdl_launch_dependents();
-    if (warp == 0) bulk_wait_all();
+    bulk_wait_all();
 }
 
-template <int kMode>
-cudaError_t launch_t(const DispatchArgs& a, cudaStream_t stream) {
-    const Geometry g = geometry(kMode, a.H);
-    const size_t smem = smem_bytes(g);
-    auto kernel = dispatch_kernel<kMode>;
+template <int kMode, int kW>
+__global__ void __launch_bounds__(32 * kW, kW == kWarps ? 2 : 1) dispatch_kernel(DispatchArgs a) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    const SliceGeo g = slice_geo(kMode, a.H);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    zero_buffer<kW>(smem, g.stage_bytes);
+    __syncthreads();
+
+    const int64_t n_tok_units = (int64_t)a.T * g.ns;
+    const int64_t stride = (int64_t)gridDim.x * kW;
+    const int64_t u = (int64_t)blockIdx.x * kW + warp;
+
+    Loads<kMode> nxt;
+    if (a.x_ready) {
+        // x is complete: load the first unit and ask L2 for the next few
+        // while the layout finishes.
+        nxt = load_x<kMode>(a, g, u, n_tok_units, lane);
+        const int64_t up = u + (int64_t)(lane + 1) * stride;
+        if (lane < kPrefetchUnits && up < n_tok_units) {
+            const int t = (int)(up / g.ns), s = (int)(up - (int64_t)t * g.ns);
+            const int ne = min(kSliceElems, a.H - s * kSliceElems);
+            const size_t eb = kMode == EP_X_FP8 ? 1 : 2;  // input bytes per element
+            bulk_prefetch_l2((const char*)a.x + ((size_t)t * a.H + (size_t)s * kSliceElems) * eb,
+                             (uint32_t)(ne * eb));
+        }
+    }
+    pdl_wait();
+    if (!a.x_ready) nxt = load_x<kMode>(a, g, u, n_tok_units, lane);
+    run_units<kMode, kW>(a, g, smem, u, nxt, ld_cg(a.num_pad_rows));
+}
+
+template <int kMode, int kW>
+cudaError_t launch_w(const DispatchArgs& a, int max_ctas, cudaStream_t stream) {
+    const SliceGeo g = slice_geo(kMode, a.H);
+    const size_t smem = smem_bytes(g, kW);
+    auto kernel = dispatch_kernel<kMode, kW>;
     cudaError_t err;
     if (smem > 48 * 1024) {
         err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (err != cudaSuccess) return err;
     }
     int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, smem);
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 32 * kW, smem);
     if (err != cudaSuccess) return err;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     // Persistent grid, no larger than the work: the number of padding rows
     // is only known on the device, E*(alignment-1) bounds it.
-    const int64_t cap = (int64_t)device_sm_count() * per_sm;
-    const int64_t want = (int64_t)a.T + ((int64_t)a.max_pad_rows + 31) / 32;
+    const int64_t cap = max_ctas > 0 ? max_ctas : (int64_t)device_sm_count() * per_sm;
+    const int64_t units = (int64_t)a.T * g.ns + a.max_pad_rows;
+    const int64_t want = (units + kW - 1) / kW;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(want < 1 ? 1 : (want < cap ? want : cap)));
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(32 * kW);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -198,12 +258,21 @@ cudaError_t launch_t(const DispatchArgs& a, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    debug_launch(kW == kWarps ? "dispatch_kernel" : "dispatch_kernel(budget)", kMode, cfg);
     return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
+// Under an SM budget of n: n CTAs of kBudgetWarps warps, each the size of
+// an SM, so the grid holds at most n SMs.
+template <int kMode>
+cudaError_t launch_t(const DispatchArgs& a, cudaStream_t stream) {
+    const int budget = sm_budget();
+    return budget > 0 ? launch_w<kMode, kBudgetWarps>(a, budget, stream) : launch_w<kMode, kWarps>(a, 0, stream);
 }
 
 }  // namespace
 
-size_t dispatch_smem_bytes(ep_x_mode mode, int H) { return smem_bytes(geometry(mode, H)); }
+size_t dispatch_smem_bytes(ep_x_mode mode, int H) { return smem_bytes(slice_geo(mode, H), kBudgetWarps); }
 
 cudaError_t launch_dispatch(const DispatchArgs& a, ep_x_mode mode, cudaStream_t stream) {
     switch (mode) {

@@ -7,6 +7,7 @@
 #include <climits>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <string>
 
 #include "ep_internal.h"
@@ -14,6 +15,7 @@
 namespace {
 
 thread_local std::string g_last_error;
+thread_local int32_t g_num_sms = 0;  // SM budget of this host thread; 0 = none
 
 ep_status invalid(const char* fmt, ...) {
     char buf[512];
@@ -122,11 +124,36 @@ int device_sm_count() {
     return n;
 }
 
+void debug_launch(const char* kernel, int variant, dim3 grid, dim3 block, size_t smem, cudaStream_t stream) {
+    static const bool on = [] {
+        const char* v = getenv("EP_DEBUG");
+        return v != nullptr && v[0] != '\0' && v[0] != '0';
+    }();
+    if (!on) return;
+    fprintf(stderr, "[ep] %s<%d>: grid %u x %u x %u, block %u, smem %zu B, stream %p, sm budget %d\n", kernel,
+            variant, grid.x, grid.y, grid.z, block.x, smem, (void*)stream, sm_budget());
+}
+
+int sm_budget() {
+    const int n = g_num_sms;
+    if (n <= 0) return 0;
+    const int sms = device_sm_count();
+    return n < sms ? n : sms;
+}
+
 }  // namespace ep
 
 extern "C" {
 
 EP_API int32_t ep_abi_version(void) { return EP_ABI_VERSION; }
+
+EP_API ep_status ep_set_num_sms(int32_t num_sms) {
+    if (num_sms < 0) return invalid("num_sms must be >= 0 (got %d); 0 means every SM", num_sms);
+    g_num_sms = num_sms;
+    return ok();
+}
+
+EP_API int32_t ep_get_num_sms(void) { return g_num_sms; }
 
 EP_API const char* ep_status_string(ep_status s) {
     switch (s) {

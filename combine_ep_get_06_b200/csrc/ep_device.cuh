@@ -8,7 +8,20 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "ep.h"
+
 namespace ep {
+
+// Checked builds (EP_CHECKED defined): EP_CHECK(cond, word) evaluates an
+// invariant that the kernels' own logic already guarantees; when it fails
+// it sets EP_DEVERR_CHECK in the error word and yields false, so that the
+// caller skips the access.  Never traps.  Production builds compile it to
+// `true`.
+#ifdef EP_CHECKED
+#define EP_CHECK(cond, word) ((cond) ? true : (atomicOr((word), EP_DEVERR_CHECK), false))
+#else
+#define EP_CHECK(cond, word) true
+#endif
 
 // 16-byte load of streamed data that does not allocate in L1 (every byte
 // is read once).  Not the non-coherent path: with programmatic dependent
@@ -81,6 +94,12 @@ __device__ __forceinline__ void bulk_s2g(void* gdst, const void* ssrc, uint32_t 
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
                  "r"(smem_addr(ssrc)), "r"(bytes)
                  : "memory");
+}
+
+// Asks the TMA engine to bring [p, p + bytes) into L2 (no shared memory,
+// no completion to wait for).  p 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 // An L2 evict-last policy (createpolicy) and a store that takes one.

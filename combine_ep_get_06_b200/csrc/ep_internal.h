@@ -125,6 +125,17 @@ cudaError_t launch_mgpu_combine(const MgpuArgs& a, cudaStream_t stream);
 
 int device_sm_count();
 
+// SM budget of this host thread (ep_set_num_sms): 0 = no budget, else the
+// most SMs the dispatch and combine grids may occupy (at most the device's).
+int sm_budget();
+
+// With EP_DEBUG=1 in the environment (read once), prints a launch's kernel,
+// variant, grid, block, dynamic shared memory and stream to stderr.
+void debug_launch(const char* kernel, int variant, dim3 grid, dim3 block, size_t smem, cudaStream_t stream);
+inline void debug_launch(const char* kernel, int variant, const cudaLaunchConfig_t& c) {
+    debug_launch(kernel, variant, c.gridDim, c.blockDim, c.dynamicSmemBytes, c.stream);
+}
+
 // Records a printf-style message for ep_last_error() and returns status.
 ep_status fail(ep_status status, const char* fmt, ...);
 

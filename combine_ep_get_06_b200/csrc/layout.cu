@@ -140,7 +140,8 @@ __global__ void __launch_bounds__(kThreads) layout_assign_kernel(LayoutArgs a) {
 }
 
 template <typename K>
-cudaError_t launch(K kernel, int grid, size_t smem, cudaStream_t stream, bool pdl, const LayoutArgs& a) {
+cudaError_t launch(K kernel, const char* name, int grid, size_t smem, cudaStream_t stream, bool pdl,
+                   const LayoutArgs& a) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);
@@ -151,6 +152,7 @@ cudaError_t launch(K kernel, int grid, size_t smem, cudaStream_t stream, bool pd
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
+    debug_launch(name, a.h.num_experts, cfg);
     return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 
@@ -167,11 +169,11 @@ cudaError_t launch_layout_t(const LayoutArgs& a, cudaStream_t stream) {
         if ((err = cudaFuncSetAttribute(assign, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
             return err;
     }
-    if (a.num_chunks == 1) return launch(single, 1, smem, stream, true, a);
+    if (a.num_chunks == 1) return launch(single, "layout_single_kernel", 1, smem, stream, true, a);
     const size_t smem_count = sizeof(int) * (E + S) + sizeof(unsigned) * 2 * kThreads;
-    err = launch(layout_count_kernel<IdxT>, a.num_chunks, smem_count, stream, true, a);
+    err = launch(layout_count_kernel<IdxT>, "layout_count_kernel", a.num_chunks, smem_count, stream, true, a);
     if (err != cudaSuccess) return err;
-    return launch(assign, a.num_chunks, smem, stream, true, a);
+    return launch(assign, "layout_assign_kernel", a.num_chunks, smem, stream, true, a);
 }
 
 }  // namespace

@@ -308,6 +308,10 @@ __device__ __forceinline__ void write_rows(const LayoutArgs& a, const Smem& m, i
         const int e = m.cq_expert[q];
         const int row = m.base[e] + (q - m.lcoff[e]);
         if (row >= a.h.max_recv_rows) continue;  // flagged by slot_row
+        // the row lies in its expert's block, before its padding
+        if (!EP_CHECK(e >= 0 && e < a.h.num_experts && row >= m.off[e] && row < m.off[e] + m.cnt[e],
+                      a.h.error_word))
+            continue;
         a.h.recv_src[row] = m.cq_slot[q];
         if (a.recv_topk_idx) a.recv_topk_idx[row] = e;
         if (a.recv_topk_weights) a.recv_topk_weights[row] = m.cq_w[q];
@@ -329,6 +333,7 @@ __device__ __forceinline__ int pad_row(const Smem& m, int E, int p) {
 __device__ __forceinline__ void write_padding(const LayoutArgs& a, const Smem& m, int E, int p0, int p1) {
     for (int p = p0 + threadIdx.x; p < p1; p += blockDim.x) {
         const int row = pad_row(m, E, p);
+        if (!EP_CHECK(p >= 0 && p < m.padoff[E] && row >= 0 && row < m.off[E], a.h.error_word)) continue;
         a.h.pad_rows[p] = row;
         if (row < a.h.max_recv_rows) {
             a.h.recv_src[row] = -1;

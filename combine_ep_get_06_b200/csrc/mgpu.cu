@@ -11,28 +11,31 @@
 // first_e is the owner's row of this rank's first slot of e.  A valid slot
 // s = t*k+j with expert e, at local row slot_map[s] (alignment-1 layout,
 // ascending slots), goes to row first_e + slot_map[s] - offsets[e] of rank
-// e/(E/W).  Token-major: each x row is read and quantised once into a
-// shared-memory buffer (the item helpers of the one-GPU dispatch).  The
-// CTA then copies it with 16-byte stores to its k destinations: peers'
-// blocks through the peer table, as plain stores over NVLink.  The slot's
-// metadata goes along with it.  After the tokens, this rank's own padding
-// rows are zeroed in its own block, and CTA 0 writes its receive totals.
-// Two row buffers alternate, so one barrier per token suffices.
-//
+// e/(E/W).  Warp units, as in the one-GPU dispatch: a unit is 1024
+// elements of one token row (or one of this rank's padding rows).  The warp
+// loads and converts the slice into its shared-memory stage, then copies it
+// with 16-byte stores to the slice's k destinations: peers' blocks through
+// the peer table, as plain stores over NVLink.  The warp that takes a
+// token's first slice also writes the token's slot metadata.  Padding rows
+// are zeroed in this rank's own block, and CTA 0 writes its receive totals.
+// No barrier after the tables: warps never wait on one another.
+
 // Combine.  The one-GPU combine with rows (rank, row) from dest: y is
 // loaded from the owners' blocks.  The arithmetic is the same: fp32 FMA
 // in ascending j from +0, one bf16 rounding.
 //
 // Neither kernel waits on another GPU.  The caller's collectives order the
 // ranks' launches.
-#include "dispatch_device.cuh"
+#include "dispatch_warp.cuh"
 
 namespace ep {
 namespace {
 
-using namespace dispatch_dev;
+using namespace warp_units;
 
 constexpr int kThreads = 256;
+
+constexpr int kWarps = kThreads / 32;
 
 struct MgpuSmem {
     int* first;      // [E]
@@ -42,14 +45,12 @@ struct MgpuSmem {
     int* own_off;    // [epr]
     int* padoff;     // [epr + 1]
     char** peer;     // [W]
-    int2* dst;       // [2][kMaxTopk]
-    unsigned char* rowbuf;  // [2][row_bytes]
-    unsigned char* sclbuf;  // [2][scale_pad]
+    unsigned char* stages;  // [kWarps][stage_bytes]
 };
 
 __host__ __device__ inline size_t align16(size_t n) { return (n + 15) & ~(size_t)15; }
 
-__host__ __device__ inline size_t mgpu_smem(int E, int epr, int W, int row_bytes, int scale_pad, MgpuSmem* m,
+__host__ __device__ inline size_t mgpu_smem(int E, int epr, int W, int stage_bytes, MgpuSmem* m,
                                             unsigned char* base) {
     size_t at = 0;
     auto take = [&](size_t n) {
@@ -64,9 +65,7 @@ __host__ __device__ inline size_t mgpu_smem(int E, int epr, int W, int row_bytes
     unsigned char* own_off = take((size_t)epr * 4);
     unsigned char* padoff = take((size_t)(epr + 1) * 4);
     unsigned char* peer = take((size_t)W * sizeof(char*));
-    unsigned char* dst = take((size_t)2 * kMaxTopk * sizeof(int2));
-    unsigned char* rowbuf = take((size_t)2 * row_bytes);
-    unsigned char* sclbuf = take((size_t)2 * scale_pad);
+    unsigned char* stages = take((size_t)kWarps * stage_bytes);
     if (m != nullptr) {
         m->first = (int*)first;
         m->lofs = (int*)lofs;
@@ -75,9 +74,7 @@ __host__ __device__ inline size_t mgpu_smem(int E, int epr, int W, int row_bytes
         m->own_off = (int*)own_off;
         m->padoff = (int*)padoff;
         m->peer = (char**)peer;
-        m->dst = (int2*)dst;
-        m->rowbuf = rowbuf;
-        m->sclbuf = sclbuf;
+        m->stages = stages;
     }
     return at;
 }
@@ -152,42 +149,48 @@ __device__ __forceinline__ int local_expert_of_pad(const MgpuSmem& m, int epr, i
     return lo;
 }
 
-// Copies n bytes from shared memory to global memory in units of 16, 4
-// or 1 bytes (the largest that divides n; the destination is aligned to it).
-__device__ __forceinline__ void copy_out(char* dst, const unsigned char* src, int n, int i0, int step) {
-    if ((n & 15) == 0) {
-        for (int i = i0; i < n / 16; i += step)
+// The lanes of a warp copy n bytes from shared memory (16-byte aligned) to
+// global memory, in the widest units that divide both n and the
+// destination's alignment.
+__device__ __forceinline__ void warp_copy_out(char* dst, const unsigned char* src, int n, int lane) {
+    const uintptr_t al = (uintptr_t)dst;
+    if ((n & 15) == 0 && (al & 15) == 0) {
+        for (int i = lane; i < n / 16; i += 32)
             reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(src)[i];
-    } else if ((n & 3) == 0) {
-        for (int i = i0; i < n / 4; i += step)
+    } else if ((n & 3) == 0 && (al & 3) == 0) {
+        for (int i = lane; i < n / 4; i += 32)
             reinterpret_cast<uint32_t*>(dst)[i] = reinterpret_cast<const uint32_t*>(src)[i];
     } else {
-        for (int i = i0; i < n; i += step) dst[i] = (char)src[i];
+        for (int i = lane; i < n; i += 32) dst[i] = (char)src[i];
     }
 }
 
-__device__ __forceinline__ void zero_out(char* dst, int n, int i0, int step) {
-    if ((n & 15) == 0) {
-        for (int i = i0; i < n / 16; i += step) reinterpret_cast<uint4*>(dst)[i] = make_uint4(0, 0, 0, 0);
-    } else if ((n & 3) == 0) {
-        for (int i = i0; i < n / 4; i += step) reinterpret_cast<uint32_t*>(dst)[i] = 0u;
+__device__ __forceinline__ void warp_zero_out(char* dst, int n, int lane) {
+    const uintptr_t al = (uintptr_t)dst;
+    if ((n & 15) == 0 && (al & 15) == 0) {
+        for (int i = lane; i < n / 16; i += 32) reinterpret_cast<uint4*>(dst)[i] = make_uint4(0, 0, 0, 0);
+    } else if ((n & 3) == 0 && (al & 3) == 0) {
+        for (int i = lane; i < n / 4; i += 32) reinterpret_cast<uint32_t*>(dst)[i] = 0u;
     } else {
-        for (int i = i0; i < n; i += step) dst[i] = 0;
+        for (int i = lane; i < n; i += 32) dst[i] = 0;
     }
 }
 
 template <int kMode>
-__global__ void __launch_bounds__(kThreads) mgpu_dispatch_kernel(MgpuArgs a) {
+__global__ void __launch_bounds__(kThreads, 3) mgpu_dispatch_kernel(MgpuArgs a) {
+    using M = Mode<kMode>;
     extern __shared__ __align__(128) unsigned char smem[];
     const ep_mgpu_geometry& g = a.g;
-    const Geometry geo = geometry(kMode, g.hidden);
+    const SliceGeo sg = slice_geo(kMode, g.hidden);
     MgpuSmem m;
-    mgpu_smem(g.num_experts, g.experts_per_rank, g.world, geo.row_bytes, geo.scale_pad, &m, smem);
+    mgpu_smem(g.num_experts, g.experts_per_rank, g.world, sg.stage_bytes, &m, smem);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int T = a.T, k = g.num_topk, epr = g.experts_per_rank;
-    const int rb_bytes = geo.row_bytes, sc_bytes = geo.scale_bytes;
+    const int rb_bytes = g.row_bytes, sc_bytes = g.scale_bytes;
     uint32_t* const err = (uint32_t*)(a.local_block + g.off_error_word);
     int2* const dest = (int2*)(a.local_block + g.off_dest);
+    unsigned char* const st = m.stages + (size_t)warp * sg.stage_bytes;
+    unsigned char* const sst = st + sg.out_bytes;
 
     build_tables(a, m);
     const int n_pad = m.padoff[epr];
@@ -207,21 +210,21 @@ __global__ void __launch_bounds__(kThreads) mgpu_dispatch_kernel(MgpuArgs a) {
         }
     }
 
-    int it = 0;
-    for (int u = blockIdx.x; u < T + n_pad; u += gridDim.x) {
-        if (u >= T) {
+    const int64_t n_tok_units = (int64_t)T * sg.ns;
+    const int64_t n_units = n_tok_units + n_pad;
+    for (int64_t u = (int64_t)blockIdx.x * kWarps + warp; u < n_units; u += (int64_t)gridDim.x * kWarps) {
+        if (u >= n_tok_units) {
             // one of this rank's padding rows, in its own block
-            const int p = u - T;
+            const int p = (int)(u - n_tok_units);
             const int i = local_expert_of_pad(m, epr, p);
             const int row = m.own_off[i] + m.own_c[i] + (p - m.padoff[i]);
             if (row >= g.max_recv_rows) {
-                if (tid == 0) atomicOr(err, EP_DEVERR_CAPACITY);
+                if (lane == 0) atomicOr(err, EP_DEVERR_CAPACITY);
                 continue;
             }
-            zero_out(a.local_block + g.off_recv_x + (size_t)row * rb_bytes, rb_bytes, tid, kThreads);
-            if (sc_bytes > 0)
-                zero_out(a.local_block + g.off_recv_scales + (size_t)row * sc_bytes, sc_bytes, tid, kThreads);
-            if (tid == 0) {
+            warp_zero_out(a.local_block + g.off_recv_x + (size_t)row * rb_bytes, rb_bytes, lane);
+            if (sc_bytes > 0) warp_zero_out(a.local_block + g.off_recv_scales + (size_t)row * sc_bytes, sc_bytes, lane);
+            if (lane == 0) {
                 ((int32_t*)(a.local_block + g.off_recv_src))[row] = -1;
                 ((int32_t*)(a.local_block + g.off_recv_topk_idx))[row] = -1;
                 ((float*)(a.local_block + g.off_recv_topk_weights))[row] = 0.0f;
@@ -229,23 +232,26 @@ __global__ void __launch_bounds__(kThreads) mgpu_dispatch_kernel(MgpuArgs a) {
             continue;
         }
 
-        const int t = u;
-        const int buf = it & 1;
-        ++it;
-        unsigned char* rb = m.rowbuf + buf * rb_bytes;
-        float* sb = reinterpret_cast<float*>(m.sclbuf + buf * geo.scale_pad);
-        int2* dst = m.dst + buf * kMaxTopk;
-
-        if (tid < k) {
-            const size_t s = (size_t)t * k + tid;
-            const int lr = a.slot_map[s];
-            int d = -1, row = -1;
+        // A token slice: its loads first, so they fly while the routing resolves.
+        const int t = (int)(u / sg.ns), s = (int)(u - (int64_t)t * sg.ns);
+        const int ne = min(kSliceElems, g.hidden - s * kSliceElems);
+        const Loads<kMode> l = load_x<kMode>(a.src, sg, u, n_tok_units, lane);
+        Meta mt;
+        mt.row = -1;
+        mt.xs = 0.0f;
+        if (kMode == EP_X_FP8 && lane < ne / 128)
+            mt.xs = a.src.x_scales[(size_t)t * (g.hidden / 128) + s * (kSliceElems / 128) + lane];
+        int d = -1, row = -1;
+        if (lane < k) {
+            const size_t sl = (size_t)t * k + lane;
+            const int lr = a.slot_map[sl];
             if (lr >= 0) {
-                const int64_t e64 = a.idx_is_int64 ? ((const int64_t*)a.topk_idx)[s] : ((const int32_t*)a.topk_idx)[s];
+                const int64_t e64 =
+                    a.idx_is_int64 ? ((const int64_t*)a.topk_idx)[sl] : ((const int32_t*)a.topk_idx)[sl];
                 const int e = (int)e64;
                 if (e64 < 0 || e64 >= g.num_experts) {
                     // not the topk_idx the layout saw: drop the slot
-                    atomicOr(err, EP_DEVERR_BAD_TOPK_IDX);
+                    if (s == 0) atomicOr(err, EP_DEVERR_BAD_TOPK_IDX);
                 } else {
                     d = e / epr;
                     row = m.first[e] + (lr - m.lofs[e]);
@@ -253,33 +259,30 @@ __global__ void __launch_bounds__(kThreads) mgpu_dispatch_kernel(MgpuArgs a) {
                 if (d < 0) {
                     row = -1;
                 } else if (row < 0 || row >= g.max_recv_rows) {
-                    atomicOr(err, EP_DEVERR_CAPACITY);
+                    if (s == 0) atomicOr(err, EP_DEVERR_CAPACITY);
                     d = row = -1;
-                } else {
+                } else if (s == 0) {
                     char* pb = m.peer[d];
-                    ((int32_t*)(pb + g.off_recv_src))[row] = (int32_t)((int64_t)g.rank * g.max_tokens * k + s);
+                    ((int32_t*)(pb + g.off_recv_src))[row] = (int32_t)((int64_t)g.rank * g.max_tokens * k + sl);
                     ((int32_t*)(pb + g.off_recv_topk_idx))[row] = e;
-                    ((float*)(pb + g.off_recv_topk_weights))[row] = a.topk_weights ? a.topk_weights[s] : 0.0f;
+                    ((float*)(pb + g.off_recv_topk_weights))[row] = a.topk_weights ? a.topk_weights[sl] : 0.0f;
                 }
             }
-            dst[tid] = make_int2(d, row);
-            dest[s] = make_int2(d, row);
+            if (s == 0) dest[sl] = make_int2(d, row);
         }
-        for (int c0 = warp * 32; c0 < geo.ipr; c0 += kThreads) {
-            const int c = c0 + lane;
-            fill_item<kMode>(a.src, t, c, c < geo.ipr, load_item<kMode>(a.src, t, c, c < geo.ipr), rb, sb);
-        }
-        __syncthreads();
-
-        // k destinations; each takes the CTA's threads in turn
+        __syncwarp();  // the previous unit's copies have read the stage
+        fill_stage<kMode>(l, mt, ne, lane, st, sst);
+        __syncwarp();
+        const int db = ne * sg.out_bytes / kSliceElems;
+        const int sb = M::kScales ? ne / M::kScaleBlock * M::kScaleBytes : 0;
         for (int j = 0; j < k; ++j) {
-            const int2 dr = dst[j];
-            if (dr.x < 0) continue;
-            char* pb = m.peer[dr.x];
-            copy_out(pb + g.off_recv_x + (size_t)dr.y * rb_bytes, rb, rb_bytes, tid, kThreads);
-            if (sc_bytes > 0)
-                copy_out(pb + g.off_recv_scales + (size_t)dr.y * sc_bytes, (const unsigned char*)sb, sc_bytes,
-                         tid, kThreads);
+            const int dj = __shfl_sync(0xffffffffu, d, j), rj = __shfl_sync(0xffffffffu, row, j);
+            if (dj < 0) continue;
+            char* pb = m.peer[dj];
+            warp_copy_out(pb + g.off_recv_x + (size_t)rj * rb_bytes + (size_t)s * sg.out_bytes, st, db, lane);
+            if (sb > 0)
+                warp_copy_out(pb + g.off_recv_scales + (size_t)rj * sc_bytes + (size_t)s * sg.sout_bytes, sst, sb,
+                              lane);
         }
     }
     // The CTA's stores to peers' memory are ordered before the grid's end:
@@ -360,9 +363,8 @@ __global__ void __launch_bounds__(kThreads) mgpu_combine_kernel(MgpuArgs a, int 
 
 template <int kMode>
 cudaError_t launch_dispatch_t(const MgpuArgs& a, cudaStream_t stream) {
-    const Geometry geo = geometry(kMode, a.g.hidden);
-    const size_t smem =
-        mgpu_smem(a.g.num_experts, a.g.experts_per_rank, a.g.world, geo.row_bytes, geo.scale_pad, nullptr, nullptr);
+    const SliceGeo sg = slice_geo(kMode, a.g.hidden);
+    const size_t smem = mgpu_smem(a.g.num_experts, a.g.experts_per_rank, a.g.world, sg.stage_bytes, nullptr, nullptr);
     auto kernel = mgpu_dispatch_kernel<kMode>;
     cudaError_t err;
     if (smem > 48 * 1024) {
@@ -374,8 +376,10 @@ cudaError_t launch_dispatch_t(const MgpuArgs& a, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int64_t cap = (int64_t)device_sm_count() * per_sm;
-    const int64_t want = (int64_t)a.T + (int64_t)a.g.experts_per_rank * (a.g.expert_alignment - 1);
+    const int64_t units = (int64_t)a.T * sg.ns + (int64_t)a.g.experts_per_rank * (a.g.expert_alignment - 1);
+    const int64_t want = (units + kWarps - 1) / kWarps;
     const int64_t grid = want < 1 ? 1 : (want < cap ? want : cap);
+    debug_launch("mgpu_dispatch_kernel", kMode, dim3((unsigned)grid), dim3(kThreads), smem, stream);
     kernel<<<(unsigned)grid, kThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
@@ -398,6 +402,7 @@ cudaError_t launch_combine_t(const MgpuArgs& a, cudaStream_t stream) {
     const int64_t cap = (int64_t)device_sm_count() * per_sm;
     const int64_t want = (int64_t)a.T * upr;
     const int64_t grid = want < 1 ? 1 : (want < cap ? want : cap);
+    debug_launch("mgpu_combine_kernel", G, dim3((unsigned)grid), dim3(bd), 0, stream);
     mgpu_combine_kernel<G><<<(unsigned)grid, bd, 0, stream>>>(a, ipr, upr);
     return cudaGetLastError();
 }
@@ -405,8 +410,8 @@ cudaError_t launch_combine_t(const MgpuArgs& a, cudaStream_t stream) {
 }  // namespace
 
 size_t mgpu_dispatch_smem_bytes(const ep_mgpu_geometry& g) {
-    const Geometry geo = geometry(g.x_mode, g.hidden);
-    return mgpu_smem(g.num_experts, g.experts_per_rank, g.world, geo.row_bytes, geo.scale_pad, nullptr, nullptr);
+    const SliceGeo sg = slice_geo(g.x_mode, g.hidden);
+    return mgpu_smem(g.num_experts, g.experts_per_rank, g.world, sg.stage_bytes, nullptr, nullptr);
 }
 
 cudaError_t launch_mgpu_dispatch(const MgpuArgs& a, ep_x_mode mode, cudaStream_t stream) {

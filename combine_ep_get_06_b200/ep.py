@@ -24,7 +24,7 @@ from . import build as _build
 
 EP_OK, EP_ERR_INVALID_ARG, EP_ERR_DEVICE, EP_ERR_CUDA = 0, 1, 2, 3
 EP_X_BF16, EP_X_FP8, EP_X_BF16_TO_FP8, EP_X_BF16_TO_NVFP4 = 0, 1, 2, 3
-EP_DEVERR_BAD_TOPK_IDX, EP_DEVERR_CAPACITY, EP_DEVERR_TIMEOUT = 1, 2, 4
+EP_DEVERR_BAD_TOPK_IDX, EP_DEVERR_CAPACITY, EP_DEVERR_TIMEOUT, EP_DEVERR_CHECK = 1, 2, 4, 8
 
 
 class EPError(RuntimeError):
@@ -64,6 +64,8 @@ SIGNATURES = {
     "ep_abi_version": (_I32, []),
     "ep_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "ep_last_error": (ctypes.c_char_p, []),
+    "ep_set_num_sms": (ctypes.c_int, [_I32]),
+    "ep_get_num_sms": (_I32, []),
     "ep_max_recv_rows": (_I32, [_I32, _I32, _I32, _I32]),
     "ep_handle_bytes": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32]),
     "ep_handle_init": (ctypes.c_int, [_HP, _I32, _I32, _I32, _I32, _I32, _I32, _P, _SZ]),
@@ -94,27 +96,67 @@ SIGNATURES = {
 }
 
 
+def _checked() -> bool:
+    """EP_CHECKED=1 in the environment selects the checked build."""
+    return os.environ.get("EP_CHECKED", "0") not in ("", "0")
+
+
 def library_path() -> str:
-    return _build.LIB
+    return _build.CHECKED_LIB if _checked() else _build.LIB
 
 
 def lib() -> ctypes.CDLL:
     """The loaded CUDA library; builds it first if the sources are newer."""
     global _LIB
     if _LIB is None:
-        if not _build.up_to_date():
+        checked = _checked()
+        path = library_path()
+        if not _build.up_to_date(checked):
             try:
-                _build.build()
+                _build.build(checked=checked)
             except Exception as exc:  # no toolkit: fail loudly, there is no fallback
-                if not os.path.exists(_build.LIB):
-                    raise RuntimeError(f"libep_b200.so is not built and cannot be built: {exc}")
-        L = ctypes.CDLL(_build.LIB)
+                if not os.path.exists(path):
+                    raise RuntimeError(f"{os.path.basename(path)} is not built and cannot be built: {exc}")
+        L = ctypes.CDLL(path)
         for name, (res, args) in SIGNATURES.items():
             fn = getattr(L, name)
             fn.restype = res
             fn.argtypes = args
         _LIB = L
     return _LIB
+
+
+def set_num_sms(num_sms: int) -> None:
+    """SM budget of this host thread (DeepEP V2 README, "Interfaces and
+    examples": num_sms): the dispatch and combine kernels launched from now
+    on occupy at most num_sms SMs, leaving the rest to a kernel running
+    beside them on another stream.  0 (the default) lets them take every
+    SM."""
+    _check(lib().ep_set_num_sms(int(num_sms)), "set_num_sms")
+
+
+def get_num_sms() -> int:
+    """This host thread's SM budget (0 = none)."""
+    return int(lib().ep_get_num_sms())
+
+
+class sm_budget:
+    """Context manager: ``with ep.sm_budget(24): ...`` runs the body's
+    dispatch / combine calls on at most 24 SMs, then restores the previous
+    budget."""
+
+    def __init__(self, num_sms: int):
+        self.num_sms = int(num_sms)
+        self.prev = 0
+
+    def __enter__(self):
+        self.prev = get_num_sms()
+        set_num_sms(self.num_sms)
+        return self
+
+    def __exit__(self, *exc):
+        set_num_sms(self.prev)
+        return False
 
 
 def _check(status: int, what: str):

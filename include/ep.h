@@ -68,6 +68,7 @@ typedef enum {
 #define EP_DEVERR_BAD_TOPK_IDX 1u /* a topk_idx value outside [-1, E): slot treated as dropped */
 #define EP_DEVERR_CAPACITY 2u     /* a row index >= max_recv_rows: write skipped */
 #define EP_DEVERR_TIMEOUT 4u      /* a bounded wait gave up */
+#define EP_DEVERR_CHECK 8u        /* a checked build (EP_CHECKED) found a broken invariant: access skipped */
 
 /* Form of the x passed to ep_dispatch (DeepEP V2 README, "Interfaces and
  * examples": x is a bf16 tensor or an FP8 (data, scale_factors) tuple). */
@@ -111,6 +112,24 @@ EP_API const char* ep_status_string(ep_status status);
 
 /* Why the last call on this host thread returned an error ("" if none). */
 EP_API const char* ep_last_error(void);
+
+/* SM budget (DeepEP V2 README, "Interfaces and examples": num_sms, the
+ * SMs the communication kernels may take, so that the expert GEMMs keep
+ * the rest; "Performance": throughput at a given #SMs).  After
+ * ep_set_num_sms(n) with n > 0, the dispatch and combine kernels that this
+ * host thread launches (ep_dispatch, ep_dispatch_mn_scales,
+ * ep_layout_dispatch's dispatch, ep_combine) use at most n CTAs, each
+ * sized to fill one SM, so they occupy at most n SMs and leave the others
+ * to a kernel running beside them on another stream.  n = 0 (the default)
+ * lets them take every SM.  Budgets above the device's SM count are
+ * clipped.  The layout kernels (one CTA per 1024 slots, a few
+ * microseconds) do not follow it.  The setting belongs to the calling host
+ * thread and is read when a call launches its kernels (a captured graph
+ * keeps the grid it was captured with).  EP_ERR_INVALID_ARG for n < 0. */
+EP_API ep_status ep_set_num_sms(int32_t num_sms);
+
+/* The calling host thread's SM budget (0 = none). */
+EP_API int32_t ep_get_num_sms(void);
 
 /* Worst-case receive rows T*k + E*(a-1): the size to give recv_x, recv_src,
  * recv_topk_idx / weights and y so that any routing fits.  -1 on bad

@@ -146,3 +146,33 @@ def test_combine_rejects_bad_arguments_before_launch():
         st = L.ep_combine(ctypes.byref(h), a["y"], a["H"], a["w"], a["rw"], a["ow"], a["out"], None)
         assert st == B.EP_ERR_INVALID_ARG, kw
         assert msg in L.ep_last_error().decode(), (kw, L.ep_last_error())
+
+
+def test_sm_budget_is_a_per_thread_setting():
+    # host only: the budget is stored, read back, rejected when negative,
+    # and belongs to the calling thread
+    import threading
+    L = B.lib()
+    assert L.ep_get_num_sms() == 0
+    assert L.ep_set_num_sms(24) == B.EP_OK and L.ep_get_num_sms() == 24
+    seen = []
+    th = threading.Thread(target=lambda: seen.append(L.ep_get_num_sms()))
+    th.start(); th.join()
+    assert seen == [0]
+    assert L.ep_set_num_sms(-1) == B.EP_ERR_INVALID_ARG and L.ep_get_num_sms() == 24
+    with B.sm_budget(64):
+        assert B.get_num_sms() == 64
+    assert B.get_num_sms() == 24
+    assert L.ep_set_num_sms(0) == B.EP_OK and L.ep_get_num_sms() == 0
+
+
+def test_checked_build_exports_the_same_abi():
+    # EP_CHECKED: the debug build with device-side invariant checks compiles
+    # (nvcc cross-compiles here) and exports exactly the production ABI
+    import subprocess
+    from combine_ep_get_06_b200 import build
+    path = build.build(checked=True)
+    def exported(p):
+        out = subprocess.run(["nm", "-D", "--defined-only", p], capture_output=True, text=True).stdout
+        return {line.split()[-1] for line in out.splitlines() if line.split()[-1].startswith("ep_")}
+    assert exported(path) == exported(build.build()) == set(B.SIGNATURES)

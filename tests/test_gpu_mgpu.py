@@ -247,3 +247,13 @@ def test_many_ranks_large_topk(world, E, k):
     # blocks hold world * max_tokens * k rows each: few tokens per rank when many ranks
     Ts = [8 + r % 5 for r in range(world)] if world >= 16 else [40 + 3 * r for r in range(world)]
     run_case(w, world, Ts, "bf16", seed=world + k)
+
+
+@pytest.mark.parametrize("mode,H", [("fp8", 1152), ("fp8", 384), ("prequant", 1152), ("nvfp4", 1056),
+                                    ("bf16", 1032)])
+def test_ragged_hidden_sizes(mode, H):
+    # a last slice shorter than 1024 elements, and scale rows that are not a
+    # multiple of 16 bytes (FP8 at H=1152: 36 B; NVFP4 at H=1056: 66 B), so
+    # the peer stores fall back to 4- and 1-byte units
+    w = dataclasses.replace(W.WORKLOADS["mid"], name=f"mid_h{H}", H=H, align=8)
+    run_case(w, 4, [200, 77, 150, 33], mode, seed=H)
