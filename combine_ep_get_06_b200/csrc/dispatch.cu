@@ -229,6 +229,224 @@ __global__ void __launch_bounds__(32 * kW, kW == kWarps ? 2 : 1) dispatch_kernel
     run_units<kMode, kW>(a, g, smem, u, nxt, ld_cg(a.num_pad_rows));
 }
 
+// --------------------------------------------------------------- row path
+//
+// Small batches (at most one layout chunk of slots, e.g. decode): a CTA
+// takes whole token rows.  Each lane converts items of 16 consecutive
+// elements (8 in bf16) into one shared row buffer -- a 1x128 block is 8
+// lanes (3 shuffles), an NVFP4 block one lane -- so a row of hidden 7168
+// takes two rounds of the CTA's threads.  After a barrier lanes j < k of
+// warp 0 copy the whole row, and its scale row, to the k receive rows with
+// one bulk copy each.  A decode launch (T=128, hidden 7168, FP8) took
+// 4.19 us in warp units, whose copies are seven times as many and a seventh
+// of the size.  Padding rows go one thread per row, slice by slice from a
+// zeroed buffer.
+constexpr int kRowWarps = 8;
+constexpr int kRowThreads = 32 * kRowWarps;
+constexpr size_t kRowSmemMax = 96 * 1024;
+
+template <int kMode>
+struct RowItem {
+    static constexpr int kElems = kMode == EP_X_BF16 ? 8 : 16;  // elements of an item
+    static constexpr bool kTwoLoads = kMode == EP_X_BF16_TO_FP8 || kMode == EP_X_BF16_TO_NVFP4;  // 32 B of bf16
+};
+
+struct Item2 {
+    uint4 v0, v1;
+};
+
+template <int kMode>
+__device__ __forceinline__ Item2 row_load(const DispatchArgs& a, int t, int c, bool active) {
+    Item2 it;
+    it.v0 = it.v1 = make_uint4(0, 0, 0, 0);
+    if (!active) return it;
+    const size_t eb = kMode == EP_X_FP8 ? 1 : 2;  // input bytes per element
+    const char* src = (const char*)a.x + ((size_t)t * a.H + (size_t)c * RowItem<kMode>::kElems) * eb;
+    it.v0 = ld_stream(src);
+    if (RowItem<kMode>::kTwoLoads) it.v1 = ld_stream(src + 16);
+    return it;
+}
+
+// Converts item c of token t into the row buffer (and its block's scale
+// into the scale buffer).  All 32 lanes of a warp call it together.
+template <int kMode>
+__device__ __forceinline__ void row_fill(const DispatchArgs& a, int t, int c, bool active, const Item2& it,
+                                         unsigned char* rowbuf, unsigned char* sclbuf) {
+    if (kMode == EP_X_BF16 || kMode == EP_X_FP8) {
+        if (active) {
+            reinterpret_cast<uint4*>(rowbuf)[c] = it.v0;
+            if (kMode == EP_X_FP8 && (c & 7) == 0)
+                reinterpret_cast<float*>(sclbuf)[c >> 3] = ld_cg(a.x_scales + (size_t)t * (a.H / 128) + (c >> 3));
+        }
+        return;
+    }
+    float f[16];
+    unpack8(it.v0, f);
+    unpack8(it.v1, f + 8);
+    float amax = fmaxf(amax8(f), amax8(f + 8));
+    if (kMode == EP_X_BF16_TO_FP8) {
+        // a 1x128 block is 8 lanes (all active or all inactive: H % 128 == 0)
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+        float scale, inv;
+        fp8_scale(amax, scale, inv);
+        const uint4 q = make_uint4(e4m3x4(f, inv), e4m3x4(f + 4, inv), e4m3x4(f + 8, inv), e4m3x4(f + 12, inv));
+        if (active) {
+            reinterpret_cast<uint4*>(rowbuf)[c] = q;
+            if ((c & 7) == 0) reinterpret_cast<float*>(sclbuf)[c >> 3] = scale;
+        }
+    } else {
+        float inv;
+        const __nv_fp8_storage_t code = nvfp4_scale(amax, inv);  // the item is one 1x16 block
+        const uint2 q = make_uint2(e2m1x8(f, inv), e2m1x8(f + 8, inv));
+        if (active) {
+            reinterpret_cast<uint2*>(rowbuf)[c] = q;
+            sclbuf[c] = code;
+        }
+    }
+}
+
+__host__ __device__ inline size_t row_smem_bytes(const SliceGeo& g) {
+    return (size_t)g.ns * g.out_bytes + (size_t)g.ns * g.sout_bytes + g.stage_bytes;  // row, scales, zeros
+}
+
+template <int kMode>
+__global__ void __launch_bounds__(32 * kRowWarps) dispatch_row_kernel(DispatchArgs a) {
+    using M = Mode<kMode>;
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ int rows_s[kMaxTopk];
+    const SliceGeo g = slice_geo(kMode, a.H);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    unsigned char* const rowbuf = smem;                                   // [ns][out_bytes]
+    unsigned char* const sclbuf = smem + (size_t)g.ns * g.out_bytes;      // [ns][sout_bytes]
+    unsigned char* const zeros = sclbuf + (size_t)g.ns * g.sout_bytes;    // [stage_bytes]
+    char* const recv = (char*)a.recv_x;
+    char* const rscl = (char*)a.recv_scales;
+    const int k = a.k, T = a.T;
+    const uint64_t keep = a.scales_ld > 0 ? l2_evict_last_policy() : 0;
+    zero_buffer<kRowWarps>(zeros, g.stage_bytes);
+    __syncthreads();
+
+    // The thread's items of a row are c = warp*32 + lane + j*kRowThreads,
+    // taken two at a time with both loads issued first.  The first pair of
+    // the CTA's first row is loaded before the wait when x is already
+    // complete (directly after the layout).
+    const int ipr = a.H / RowItem<kMode>::kElems;
+    const int c0 = warp * 32;
+    Item2 fa, fb;
+    const bool first_ok = blockIdx.x < (unsigned)T;
+    if (a.x_ready && first_ok) {
+        fa = row_load<kMode>(a, blockIdx.x, c0 + lane, c0 + lane < ipr);
+        fb = row_load<kMode>(a, blockIdx.x, c0 + kRowThreads + lane, c0 + kRowThreads + lane < ipr);
+    }
+    pdl_wait();
+    if (!a.x_ready && first_ok) {
+        fa = row_load<kMode>(a, blockIdx.x, c0 + lane, c0 + lane < ipr);
+        fb = row_load<kMode>(a, blockIdx.x, c0 + kRowThreads + lane, c0 + kRowThreads + lane < ipr);
+    }
+    bool have_first = first_ok && c0 < ipr;  // used by the first pass of the loop below
+
+    const bool bulk_scl = M::kScales && a.bulk_scales;
+    for (int t = blockIdx.x; t < T; t += gridDim.x) {
+        if (tid < k) rows_s[tid] = ld_cg(a.slot_map + (size_t)t * k + tid);
+        for (int c = c0; c < ipr; c += 2 * kRowThreads) {
+            const int ca = c + lane, cb = c + kRowThreads + lane;
+            Item2 ia, ib;
+            if (have_first) {
+                ia = fa;
+                ib = fb;
+                have_first = false;
+            } else {
+                ia = row_load<kMode>(a, t, ca, ca < ipr);
+                ib = row_load<kMode>(a, t, cb, cb < ipr);
+            }
+            row_fill<kMode>(a, t, ca, ca < ipr, ia, rowbuf, sclbuf);
+            if (c + kRowThreads < ipr) row_fill<kMode>(a, t, cb, cb < ipr, ib, rowbuf, sclbuf);
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (warp == 0 && lane < k) {
+            const int row = rows_s[lane];
+            if (row >= 0 && row < a.max_rows) {
+                bulk_s2g(recv + (size_t)row * g.row_bytes, rowbuf, g.row_bytes);
+                if (bulk_scl) bulk_s2g(rscl + (size_t)row * g.srow_bytes, sclbuf, g.srow_bytes);
+            } else if (row >= a.max_rows) {
+                atomicOr(a.error_word, EP_DEVERR_CAPACITY);
+            }
+            bulk_commit();
+            bulk_wait_read<0>();  // the buffer is refilled after the barrier below
+        }
+        if (M::kScales && !bulk_scl) {
+            // MN-major scales, or scale rows that are not a multiple of 16 bytes: plain stores.
+            const int B = a.H / M::kScaleBlock;
+            for (int i = tid; i < k * B; i += blockDim.x) {
+                const int row = rows_s[i / B];
+                if (row >= 0 && row < a.max_rows) store_scale<kMode>(a, row, i % B, sclbuf, i % B, keep);
+            }
+        }
+        __syncthreads();
+    }
+
+    const int n_pad = ld_cg(a.num_pad_rows);
+    for (int p = blockIdx.x * blockDim.x + tid; p < n_pad; p += gridDim.x * blockDim.x) {
+        const int row = ld_cg(a.pad_rows + p);
+        if (row < 0 || row >= a.max_rows) {
+            if (row >= a.max_rows) atomicOr(a.error_word, EP_DEVERR_CAPACITY);
+            continue;
+        }
+        for (int s = 0; s < g.ns; ++s) {
+            const int ne = min(kSliceElems, a.H - s * kSliceElems);
+            bulk_s2g(recv + (size_t)row * g.row_bytes + (size_t)s * g.out_bytes, zeros, ne * g.out_bytes / kSliceElems);
+            if (M::kScales && bulk_scales_ok<kMode>(a, ne))
+                bulk_s2g(rscl + (size_t)row * g.srow_bytes + (size_t)s * g.sout_bytes, zeros,
+                         ne / M::kScaleBlock * M::kScaleBytes);
+        }
+        bulk_commit();
+        if (M::kScales) {
+            constexpr int kPerSlice = kSliceElems / M::kScaleBlock;
+            const int B = a.H / M::kScaleBlock;
+            for (int b = 0; b < B; ++b)
+                if (!bulk_scales_ok<kMode>(a, min(kSliceElems, a.H - (b / kPerSlice) * kSliceElems)))
+                    store_scale<kMode>(a, row, b, nullptr, 0, keep);
+        }
+    }
+    pdl_launch_dependents();
+    bulk_wait_all();
+}
+
+template <int kMode>
+cudaError_t launch_row_t(const DispatchArgs& a, cudaStream_t stream) {
+    const SliceGeo g = slice_geo(kMode, a.H);
+    const size_t smem = row_smem_bytes(g);
+    auto kernel = dispatch_row_kernel<kMode>;
+    cudaError_t err;
+    if (smem > 48 * 1024) {
+        err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err != cudaSuccess) return err;
+    }
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 32 * kRowWarps, smem);
+    if (err != cudaSuccess) return err;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int64_t cap = (int64_t)device_sm_count() * per_sm;
+    int64_t want = a.T;
+    const int64_t pad_ctas = ((int64_t)a.max_pad_rows + 32 * kRowWarps - 1) / (32 * kRowWarps);
+    if (pad_ctas > want) want = pad_ctas;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(want < 1 ? 1 : (want < cap ? want : cap)));
+    cfg.blockDim = dim3(32 * kRowWarps);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    debug_launch("dispatch_row_kernel", kMode, cfg);
+    return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
 template <int kMode, int kW>
 cudaError_t launch_w(const DispatchArgs& a, int max_ctas, cudaStream_t stream) {
     const SliceGeo g = slice_geo(kMode, a.H);
@@ -263,11 +481,15 @@ cudaError_t launch_w(const DispatchArgs& a, int max_ctas, cudaStream_t stream) {
 }
 
 // Under an SM budget of n: n CTAs of kBudgetWarps warps, each the size of
-// an SM, so the grid holds at most n SMs.
+// an SM, so the grid holds at most n SMs.  Without one, batches of at most
+// one layout chunk of slots take the row path.
 template <int kMode>
 cudaError_t launch_t(const DispatchArgs& a, cudaStream_t stream) {
     const int budget = sm_budget();
-    return budget > 0 ? launch_w<kMode, kBudgetWarps>(a, budget, stream) : launch_w<kMode, kWarps>(a, 0, stream);
+    if (budget > 0) return launch_w<kMode, kBudgetWarps>(a, budget, stream);
+    if ((int64_t)a.T * a.k <= kLayoutChunkSlots && row_smem_bytes(slice_geo(kMode, a.H)) <= kRowSmemMax)
+        return launch_row_t<kMode>(a, stream);
+    return launch_w<kMode, kWarps>(a, 0, stream);
 }
 
 }  // namespace

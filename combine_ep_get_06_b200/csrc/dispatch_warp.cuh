@@ -99,6 +99,55 @@ __device__ __forceinline__ Loads<kMode> load_x(const DispatchArgs& a, const Slic
     return l;
 }
 
+// ---- conversions shared by the warp units and the row path
+
+// bf16 pairs (low half first) of four 32-bit words -> 8 floats, exactly.
+__device__ __forceinline__ void unpack8(const uint4& v, float* f) {
+    f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x); f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+    f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z); f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+}
+
+// FP8 block scale from the block's amax: scale = amax/448 and inv = 448/amax
+// (amax floored at 1e-4), each one IEEE division.
+__device__ __forceinline__ void fp8_scale(float amax, float& scale, float& inv) {
+    amax = fmaxf(amax, kAmaxFloor);
+    scale = __fdiv_rn(amax, kE4m3Max);
+    inv = __fdiv_rn(kE4m3Max, amax);
+}
+
+// 4 floats times inv (one rounding each) -> 4 e4m3 bytes, nearest-even, saturating.
+__device__ __forceinline__ uint32_t e4m3x4(const float* f, float inv) {
+    return pack_e4m3x2(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv)) |
+           (pack_e4m3x2(__fmul_rn(f[2], inv), __fmul_rn(f[3], inv)) << 16);
+}
+
+// NVFP4 block scale from the 1x16 block's amax (floored at 6*2^-9): the
+// e4m3 code of amax/6 and the inverse of the decoded scale.
+__device__ __forceinline__ __nv_fp8_storage_t nvfp4_scale(float amax, float& inv) {
+    amax = fmaxf(amax, kFp4AmaxFloor);
+    const __nv_fp8_storage_t code = __nv_cvt_float_to_fp8(__fdiv_rn(amax, kE2m1Max), __NV_SATFINITE, __NV_E4M3);
+    inv = __fdiv_rn(1.0f, __half2float(__half(__nv_cvt_fp8_to_halfraw(code, __NV_E4M3))));
+    return code;
+}
+
+// 8 floats times inv -> 8 E2M1 codes in 4 bytes, the even element in the low nibble.
+__device__ __forceinline__ uint32_t e2m1x8(const float* f, float inv) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+        w |= (uint32_t)__nv_cvt_float2_to_fp4x2(make_float2(__fmul_rn(f[2 * e], inv), __fmul_rn(f[2 * e + 1], inv)),
+                                                 __NV_E2M1, cudaRoundNearest)
+             << (8 * e);
+    return w;
+}
+
+__device__ __forceinline__ float amax8(const float* f) {
+    float m = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
+    return m;
+}
+
 // Converts the unit's loads into the stage: data at st, scales at sst.
 template <int kMode>
 __device__ __forceinline__ void fill_stage(const Loads<kMode>& l, const Meta& m, int ne, int lane,
@@ -112,22 +161,16 @@ __device__ __forceinline__ void fill_stage(const Loads<kMode>& l, const Meta& m,
         if (kMode == EP_X_BF16 || kMode == EP_X_FP8) {
             if (active) reinterpret_cast<uint4*>(st)[idx] = v;
         } else {
-            const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
-                                bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
-            float amax = 0.0f;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+            float f[8];
+            unpack8(v, f);
+            float amax = amax8(f);
             if (kMode == EP_X_BF16_TO_FP8) {
                 // a 1x128 block is 16 lanes (all active or all inactive: H % 128 == 0)
 #pragma unroll
                 for (int o = 1; o < 16; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-                amax = fmaxf(amax, kAmaxFloor);
-                const float scale = __fdiv_rn(amax, kE4m3Max);
-                const float inv = __fdiv_rn(kE4m3Max, amax);
-                const uint32_t w0 = pack_e4m3x2(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv)) |
-                                    (pack_e4m3x2(__fmul_rn(f[2], inv), __fmul_rn(f[3], inv)) << 16);
-                const uint32_t w1 = pack_e4m3x2(__fmul_rn(f[4], inv), __fmul_rn(f[5], inv)) |
-                                    (pack_e4m3x2(__fmul_rn(f[6], inv), __fmul_rn(f[7], inv)) << 16);
+                float scale, inv;
+                fp8_scale(amax, scale, inv);
+                const uint32_t w0 = e4m3x4(f, inv), w1 = e4m3x4(f + 4, inv);
                 if (active) {
                     reinterpret_cast<uint2*>(st)[idx] = make_uint2(w0, w1);
                     if ((lane & 15) == 0) reinterpret_cast<float*>(sst)[idx >> 4] = scale;
@@ -135,18 +178,9 @@ __device__ __forceinline__ void fill_stage(const Loads<kMode>& l, const Meta& m,
             } else {
                 // NVFP4: a 1x16 block is a lane pair (H % 32 == 0)
                 amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-                amax = fmaxf(amax, kFp4AmaxFloor);
-                const __nv_fp8_storage_t code =
-                    __nv_cvt_float_to_fp8(__fdiv_rn(amax, kE2m1Max), __NV_SATFINITE, __NV_E4M3);
-                const float scale = __half2float(__half(__nv_cvt_fp8_to_halfraw(code, __NV_E4M3)));
-                const float inv = __fdiv_rn(1.0f, scale);
-                uint32_t w = 0;
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    w |= (uint32_t)__nv_cvt_float2_to_fp4x2(
-                             make_float2(__fmul_rn(f[2 * e], inv), __fmul_rn(f[2 * e + 1], inv)), __NV_E2M1,
-                             cudaRoundNearest)
-                         << (8 * e);
+                float inv;
+                const __nv_fp8_storage_t code = nvfp4_scale(amax, inv);
+                const uint32_t w = e2m1x8(f, inv);
                 if (active) {
                     reinterpret_cast<uint32_t*>(st)[idx] = w;
                     if ((lane & 1) == 0) sst[idx >> 1] = code;

@@ -36,6 +36,7 @@ using namespace warp_units;
 constexpr int kThreads = 256;
 
 constexpr int kWarps = kThreads / 32;
+constexpr int kMinUnitsPerWarp = 8;
 
 struct MgpuSmem {
     int* first;      // [E]
@@ -375,9 +376,14 @@ cudaError_t launch_dispatch_t(const MgpuArgs& a, cudaStream_t stream) {
     err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, smem);
     if (err != cudaSuccess) return err;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    // Every CTA first builds its tables from the gathered counts (W x E
+    // loads and scans): give each warp at least kMinUnitsPerWarp units so
+    // that this set-up is amortised (measured with 8 ranks of 1024 tokens on
+    // one GPU: 204 -> 180 us for the dispatch phase); large batches still
+    // fill every SM.
     const int64_t cap = (int64_t)device_sm_count() * per_sm;
     const int64_t units = (int64_t)a.T * sg.ns + (int64_t)a.g.experts_per_rank * (a.g.expert_alignment - 1);
-    const int64_t want = (units + kWarps - 1) / kWarps;
+    const int64_t want = (units + kWarps * kMinUnitsPerWarp - 1) / (kWarps * kMinUnitsPerWarp);
     const int64_t grid = want < 1 ? 1 : (want < cap ? want : cap);
     debug_launch("mgpu_dispatch_kernel", kMode, dim3((unsigned)grid), dim3(kThreads), smem, stream);
     kernel<<<(unsigned)grid, kThreads, smem, stream>>>(a);
