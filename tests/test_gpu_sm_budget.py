@@ -80,9 +80,10 @@ def _time(fn, n=10):
     return a.elapsed_time(b) / n
 
 
-@pytest.mark.parametrize("budget", [24, 64])
-def test_budget_results_match_oracle(budget):
-    c = Case("mid")
+@pytest.mark.parametrize("name,budget", [("mid", 24), ("mid", 64), ("decode", 16)])
+def test_budget_results_match_oracle(name, budget):
+    # decode-sized batches take the row path without a budget, warp units with one
+    c = Case(name)
     with ep.sm_budget(budget):
         c.step()
     assert ep.get_num_sms() == 0
