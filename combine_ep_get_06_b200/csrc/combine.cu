@@ -102,11 +102,18 @@ __global__ void __launch_bounds__(kMaxT) combine_kernel(CombineArgs a, int ipr, 
     pdl_launch_dependents();
 }
 
-int unit_threads(int ipr) {
-    for (int bd = kMaxThreads; bd >= 32; bd -= 32)
+// Threads of a unit: the largest multiple of 32 up to `most` that divides
+// the row's items, else the row rounded up to a warp (or `most`).
+int unit_threads(int ipr, int most) {
+    for (int bd = most; bd >= 32; bd -= 32)
         if (ipr % bd == 0) return bd;
-    return ipr < kMaxThreads ? ((ipr + 31) / 32) * 32 : kMaxThreads;
+    return ipr < most ? ((ipr + 31) / 32) * 32 : most;
 }
+
+// Below this many units per SM a batch is one short wave (decode sizes):
+// units of at most 128 threads then spread its rows over more CTAs, so
+// that every SM gets a similar share of the row loads.
+constexpr int kSmallUnitsPerSm = 8;
 
 template <int G, int kMaxT>
 cudaError_t launch_bd(const CombineArgs& a, int ipr, int ut, int bd, int max_ctas, cudaStream_t stream) {
@@ -142,8 +149,10 @@ cudaError_t launch_bd(const CombineArgs& a, int ipr, int ut, int bd, int max_cta
 template <int G>
 cudaError_t launch_t(const CombineArgs& a, cudaStream_t stream) {
     const int ipr = a.H / 8;
-    const int ut = unit_threads(ipr);
+    int ut = unit_threads(ipr, kMaxThreads);
     const int budget = sm_budget();
+    if (budget == 0 && (int64_t)a.T * ((ipr + ut - 1) / ut) < (int64_t)kSmallUnitsPerSm * device_sm_count())
+        ut = unit_threads(ipr, 128);
     if (budget > 0) {
         constexpr int kT = budget_threads<G>();
         return launch_bd<G, kT>(a, ipr, ut, (kT / ut) * ut, budget, stream);

@@ -18,12 +18,21 @@
 // cycles kStages stages: a stage is refilled only once the copies issued
 // from it kStages units ago have read it.
 //
+// Three launch shapes share the per-unit code (dispatch_warp.cuh):
+//   - warp units, 8-warp CTAs, 2 to an SM (the default);
+//   - under an SM budget of n (ep_set_num_sms), warp units in n CTAs of 24
+//     warps, each CTA filling an SM;
+//   - batches of at most one layout chunk of slots (e.g. decode): the row
+//     path, a CTA per token row with one bulk copy per destination row (see
+//     the row path below).
+//
 // Launched with programmatic dependent launch: the first unit's x loads
 // may be issued before waiting for the previous grid (only directly after
 // the layout, which leaves x untouched), everything the layout writes is
 // read after the wait, and the next grid may start launching once all
 // copies are issued.
 #include "dispatch_warp.cuh"
+#include "layout_device.cuh"
 
 namespace ep {
 namespace {
@@ -243,6 +252,7 @@ __global__ void __launch_bounds__(32 * kW, kW == kWarps ? 2 : 1) dispatch_kernel
 // zeroed buffer.
 constexpr int kRowWarps = 8;
 constexpr int kRowThreads = 32 * kRowWarps;
+static_assert(kLayoutChunkSlots % kRowThreads == 0, "a one-chunk layout spreads evenly over a row CTA");
 constexpr size_t kRowSmemMax = 96 * 1024;
 
 template <int kMode>
@@ -311,8 +321,271 @@ __host__ __device__ inline size_t row_smem_bytes(const SliceGeo& g) {
     return (size_t)g.ns * g.out_bytes + (size_t)g.ns * g.sout_bytes + g.stage_bytes;  // row, scales, zeros
 }
 
-template <int kMode>
-__global__ void __launch_bounds__(32 * kRowWarps) dispatch_row_kernel(DispatchArgs a) {
+// ---- the layout inside every CTA (one-chunk batches through ep_layout_dispatch)
+//
+// With at most kLayoutChunkSlots slots there is no layout grid.  Every CTA
+// reads all T*k expert indices into shared memory and computes what it
+// needs: the per-expert counts (shared atomics), the aligned expert offsets
+// (a scan over the experts), and, for each slot of its own tokens, the
+// number of earlier slots with the same expert (ballot counts over the
+// index array), which gives the slot's row.  It writes the handle entries
+// of its own slots and of the padding rows it zeroes; CTA 0 also writes the
+// totals and the tokens per segment.  No CTA waits for another.
+
+// Shared memory of the in-CTA layout, after the row buffers.
+struct RowLayout {
+    int* eidx;    // [T*k] expert of each slot, -1 when dropped
+    int* cnt;     // [E]   slots of each expert
+    int* pre;     // [E]   slots of each expert before the CTA's first token
+    int* off;     // [E+1] first row of each expert
+    int* padoff;  // [E+1] first padding index of each expert
+    int* wsum;    // [2*kRowWarps] scan of the warps' sums
+    float* w0;    // [kMaxTopk] weights of the CTA's first token's slots
+    __device__ RowLayout(int* p, int n, int E) {
+        eidx = p;
+        cnt = eidx + n;
+        pre = cnt + E;
+        off = pre + E;
+        padoff = off + E + 1;
+        wsum = padoff + E + 1;
+        w0 = reinterpret_cast<float*>(wsum + 2 * kRowWarps);
+    }
+};
+
+__host__ __device__ inline size_t row_layout_bytes(int n, int E) {
+    return sizeof(int) * ((size_t)n + 2 * (size_t)E + 2 * ((size_t)E + 1) + 2 * kRowWarps + kMaxTopk);
+}
+
+// off / padoff from cnt: aligned rows A(c) = ceil(c/a)*a and padding rows
+// A(c) - c, scanned over the experts by kRowThreads threads, each taking a
+// run of consecutive experts.  Barriers inside; ends with one.
+__device__ __forceinline__ void row_expert_offsets(const RowLayout& L, int E, int align) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int per = (E + kRowThreads - 1) / kRowThreads;
+    const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
+    int r = 0, p = 0;
+    for (int e = e0; e < e1; ++e) {
+        const int c = L.cnt[e], re = align == 1 ? c : (c + align - 1) / align * align;
+        r += re;
+        p += re - c;
+    }
+    int ri = r, pi = p;  // inclusive scan within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int ro = __shfl_up_sync(0xffffffffu, ri, o), po = __shfl_up_sync(0xffffffffu, pi, o);
+        if (lane >= o) {
+            ri += ro;
+            pi += po;
+        }
+    }
+    if (lane == 31) {
+        L.wsum[warp] = ri;
+        L.wsum[kRowWarps + warp] = pi;
+    }
+    __syncthreads();
+    int rb = ri - r, pb = pi - p;
+    for (int w = 0; w < warp; ++w) {
+        rb += L.wsum[w];
+        pb += L.wsum[kRowWarps + w];
+    }
+    for (int e = e0; e < e1; ++e) {
+        const int c = L.cnt[e], re = align == 1 ? c : (c + align - 1) / align * align;
+        L.off[e] = rb;
+        L.padoff[e] = pb;
+        rb += re;
+        pb += re - c;
+    }
+    if (tid == kRowThreads - 1) {
+        L.off[E] = rb;
+        L.padoff[E] = pb;
+    }
+    __syncthreads();
+}
+
+// Row of padding index p: the expert by binary search on padoff.
+__device__ __forceinline__ int row_pad_row(const RowLayout& L, int E, int p) {
+    int lo = 0, hi = E;  // padoff[lo] <= p < padoff[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (L.padoff[mid] <= p) lo = mid;
+        else hi = mid;
+    }
+    return L.off[lo] + L.cnt[lo] + (p - L.padoff[lo]);
+}
+
+// The in-CTA layout in two parts, so that the row conversion runs while
+// the index loads are in flight.  row_layout_load issues the loads of the
+// T*k expert indices (a thread takes kSlotsPerThread consecutive slots)
+// and of the weights of the CTA's first token, and zeroes the counts;
+// row_layout_count then (after a barrier) stores the indices, counts them
+// per expert (and before the CTA's first token), and scans the offsets.
+constexpr int kSlotsPerThread = kLayoutChunkSlots / kRowThreads;
+
+// An index load issued where it stands (a volatile asm is not moved past
+// the other volatile loads), so that it is in flight during the conversion.
+template <typename IdxT>
+__device__ __forceinline__ long long ld_idx(const IdxT* p) {
+    static_assert(sizeof(IdxT) == 8 || sizeof(IdxT) == 4, "int32 or int64 indices");
+    if constexpr (sizeof(IdxT) == 8) {
+        long long v;
+        asm volatile("ld.global.nc.s64 %0, [%1];" : "=l"(v) : "l"(p));
+        return v;
+    } else {
+        int v;
+        asm volatile("ld.global.nc.s32 %0, [%1];" : "=r"(v) : "l"(p));
+        return v;
+    }
+}
+__device__ __forceinline__ float ld_weight(const float* p) {
+    float v;
+    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
+}
+
+// Raw values (checked in row_layout_count) and, for threads below k, the
+// weight of the CTA's first token's slot tid, kept in registers until then.
+template <typename IdxT>
+__device__ __forceinline__ void row_layout_load(const LayoutArgs& la, const RowLayout& L,
+                                                long long (&ev)[kSlotsPerThread], float& w0) {
+    const int E = la.h.num_experts, n = la.h.num_tokens * la.h.num_topk;
+    const int tid = threadIdx.x;
+#pragma unroll
+    for (int r = 0; r < kSlotsPerThread; ++r) {
+        const int i = tid * kSlotsPerThread + r;
+        ev[r] = i < n ? ld_idx((const IdxT*)la.topk_idx + i) : -1;
+    }
+    w0 = 0.0f;
+    if (tid < la.h.num_topk && la.topk_weights && (int)blockIdx.x < la.h.num_tokens)
+        w0 = ld_weight(la.topk_weights + (size_t)blockIdx.x * la.h.num_topk + tid);
+    for (int e = tid; e < E; e += kRowThreads) {
+        L.cnt[e] = 0;
+        L.pre[e] = 0;
+    }
+}
+
+__device__ __forceinline__ void row_layout_count(const LayoutArgs& la, const RowLayout& L,
+                                                 const long long (&ev)[kSlotsPerThread], float w0) {
+    const int E = la.h.num_experts, n = la.h.num_tokens * la.h.num_topk;
+    const int tid = threadIdx.x;
+    if (tid < la.h.num_topk) L.w0[tid] = w0;
+    __syncthreads();  // the counts are zero
+    const int first = blockIdx.x * la.h.num_topk;  // the CTA's first slot
+    bool bad = false;
+#pragma unroll
+    for (int r = 0; r < kSlotsPerThread; ++r) {
+        const int i = tid * kSlotsPerThread + r;
+        if (i < n) {
+            // a value outside [-1, E) flags the error word and drops the slot
+            const bool ok = ev[r] >= -1 && ev[r] < E;
+            bad |= !ok;
+            const int e = ok ? (int)ev[r] : -1;
+            L.eidx[i] = e;
+            if (e >= 0) {
+                atomicAdd(&L.cnt[e], 1);
+                if (i < first) atomicAdd(&L.pre[e], 1);
+            }
+        }
+    }
+    if (bad) atomicOr(la.h.error_word, EP_DEVERR_BAD_TOPK_IDX);
+    __syncthreads();
+    row_expert_offsets(L, E, la.h.expert_alignment);
+}
+
+// The rows of token t's slots into rows_s, and their handle entries.  Slot
+// j is warp j % kRowWarps's: its row is off[e] plus the number of earlier
+// slots (flat order) with expert e.  For the CTA's first token that is
+// pre[e] plus the token's own earlier slots; for later ones (several tokens
+// to a CTA) the slots are counted 128 at a time by ballots.
+__device__ __forceinline__ void row_slots(const LayoutArgs& la, const RowLayout& L, int t, int* rows_s) {
+    const int k = la.h.num_topk, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int j = warp; j < k; j += kRowWarps) {
+        const int s = t * k + j;
+        const int e = L.eidx[s];
+        int row = -1;
+        if (e >= 0) {
+            int before = 0;
+            if (t == (int)blockIdx.x) {  // the CTA's first token: pre counts the slots before it
+                before = L.pre[e];
+                for (int jj = 0; jj < j; ++jj) before += L.eidx[t * k + jj] == e;
+            } else {
+                for (int c = 0; c < s; c += 128) {
+                    bool hit[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int i = c + 32 * q + lane;
+                        hit[q] = i < s && L.eidx[i] == e;
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) before += __popc(__ballot_sync(0xffffffffu, hit[q]));
+                }
+            }
+            row = L.off[e] + before;
+            if (row >= la.h.max_recv_rows) {
+                if (lane == 0) atomicOr(la.h.error_word, EP_DEVERR_CAPACITY);
+                row = -1;
+            } else if (lane == 0) {
+                la.h.recv_src[row] = s;
+                if (la.recv_topk_idx) la.recv_topk_idx[row] = e;
+                if (la.recv_topk_weights)
+                    la.recv_topk_weights[row] =
+                        !la.topk_weights ? 0.0f : t == (int)blockIdx.x ? L.w0[j] : __ldg(la.topk_weights + s);
+            }
+        }
+        if (lane == 0) {
+            la.h.slot_map[s] = row;
+            rows_s[j] = row;
+        }
+    }
+}
+
+// Every CTA's share of the handle totals: the per-expert arrays of experts
+// [E*b/G, E*(b+1)/G), and the token counts of segments g = b, b+G, ... (a
+// token counts once in each segment one of its valid slots reaches; block
+// sum of the threads' counts).  CTA 0 also writes offsets[E] and the
+// padding count.
+__device__ __forceinline__ void row_totals(const LayoutArgs& la, const RowLayout& L) {
+    const int E = la.h.num_experts, S = la.h.num_segments, k = la.h.num_topk, T = la.h.num_tokens;
+    const int b = blockIdx.x, G = gridDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int e0 = (int)((int64_t)E * b / G), e1 = (int)((int64_t)E * (b + 1) / G);
+    for (int e = e0 + tid; e < e1; e += kRowThreads) {
+        la.h.counts[e] = L.cnt[e];
+        la.h.recv_counts[e] = L.off[e + 1] - L.off[e];
+        la.h.offsets[e] = L.off[e];
+    }
+    if (b == 0 && tid == 0) {
+        la.h.offsets[E] = L.off[E];
+        *la.h.num_pad_rows = L.padoff[E];
+    }
+    const int per_seg = E / S;
+    for (int gs = b; gs < S; gs += G) {
+        const int lo = gs * per_seg, hi = lo + per_seg;  // the segment's experts
+        int c = 0;
+        for (int t = tid; t < T; t += kRowThreads) {
+            bool has = false;
+            for (int j = 0; j < k; ++j) {
+                const int e = L.eidx[t * k + j];
+                has |= e >= lo && e < hi;
+            }
+            c += has;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+        __syncthreads();  // wsum is free
+        if (lane == 0) L.wsum[warp] = c;
+        __syncthreads();
+        if (tid == 0) {
+            int sum = 0;
+            for (int w = 0; w < kRowWarps; ++w) sum += L.wsum[w];
+            la.h.seg_tokens[gs] = sum;
+        }
+    }
+}
+
+// The row path.  kLayout: the in-CTA layout above (launched as the first
+// grid of ep_layout_dispatch, so x too is read only after the wait);
+// otherwise the routing comes from the handle the layout grid wrote.
+template <int kMode, bool kLayout, typename IdxT>
+__global__ void __launch_bounds__(kRowThreads, 2) dispatch_row_kernel(DispatchArgs a, LayoutArgs la) {
     using M = Mode<kMode>;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ int rows_s[kMaxTopk];
@@ -321,6 +594,8 @@ __global__ void __launch_bounds__(32 * kRowWarps) dispatch_row_kernel(DispatchAr
     unsigned char* const rowbuf = smem;                                   // [ns][out_bytes]
     unsigned char* const sclbuf = smem + (size_t)g.ns * g.out_bytes;      // [ns][sout_bytes]
     unsigned char* const zeros = sclbuf + (size_t)g.ns * g.sout_bytes;    // [stage_bytes]
+    const RowLayout L(reinterpret_cast<int*>(zeros + g.stage_bytes), kLayout ? a.T * a.k : 0,
+                      kLayout ? la.h.num_experts : 0);
     char* const recv = (char*)a.recv_x;
     char* const rscl = (char*)a.recv_scales;
     const int k = a.k, T = a.T;
@@ -331,7 +606,7 @@ __global__ void __launch_bounds__(32 * kRowWarps) dispatch_row_kernel(DispatchAr
     // The thread's items of a row are c = warp*32 + lane + j*kRowThreads,
     // taken two at a time with both loads issued first.  The first pair of
     // the CTA's first row is loaded before the wait when x is already
-    // complete (directly after the layout).
+    // complete (directly after the layout grid).
     const int ipr = a.H / RowItem<kMode>::kElems;
     const int c0 = warp * 32;
     Item2 fa, fb;
@@ -346,10 +621,14 @@ __global__ void __launch_bounds__(32 * kRowWarps) dispatch_row_kernel(DispatchAr
         fb = row_load<kMode>(a, blockIdx.x, c0 + kRowThreads + lane, c0 + kRowThreads + lane < ipr);
     }
     bool have_first = first_ok && c0 < ipr;  // used by the first pass of the loop below
+    long long ev[kSlotsPerThread];
+    float w0 = 0.0f;
+    if (kLayout) row_layout_load<IdxT>(la, L, ev, w0);
+    bool laid_out = !kLayout;  // CTA-uniform
 
     const bool bulk_scl = M::kScales && a.bulk_scales;
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
-        if (tid < k) rows_s[tid] = ld_cg(a.slot_map + (size_t)t * k + tid);
+        if (!kLayout && tid < k) rows_s[tid] = ld_cg(a.slot_map + (size_t)t * k + tid);
         for (int c = c0; c < ipr; c += 2 * kRowThreads) {
             const int ca = c + lane, cb = c + kRowThreads + lane;
             Item2 ia, ib;
@@ -364,18 +643,27 @@ __global__ void __launch_bounds__(32 * kRowWarps) dispatch_row_kernel(DispatchAr
             row_fill<kMode>(a, t, ca, ca < ipr, ia, rowbuf, sclbuf);
             if (c + kRowThreads < ipr) row_fill<kMode>(a, t, cb, cb < ipr, ib, rowbuf, sclbuf);
         }
+        if (kLayout) {
+            if (!laid_out) {
+                row_layout_count(la, L, ev, w0);
+                laid_out = true;
+            }
+            row_slots(la, L, t, rows_s);
+        }
         fence_proxy_async_smem();
         __syncthreads();
-        if (warp == 0 && lane < k) {
-            const int row = rows_s[lane];
-            if (row >= 0 && row < a.max_rows) {
-                bulk_s2g(recv + (size_t)row * g.row_bytes, rowbuf, g.row_bytes);
-                if (bulk_scl) bulk_s2g(rscl + (size_t)row * g.srow_bytes, sclbuf, g.srow_bytes);
-            } else if (row >= a.max_rows) {
-                atomicOr(a.error_word, EP_DEVERR_CAPACITY);
+        if (lane == 0) {  // warp j issues the copies of slots j, j + kRowWarps, ...
+            for (int j = warp; j < k; j += kRowWarps) {
+                const int row = rows_s[j];
+                if (row >= 0 && row < a.max_rows) {
+                    bulk_s2g(recv + (size_t)row * g.row_bytes, rowbuf, g.row_bytes);
+                    if (bulk_scl) bulk_s2g(rscl + (size_t)row * g.srow_bytes, sclbuf, g.srow_bytes);
+                } else if (row >= a.max_rows) {
+                    atomicOr(a.error_word, EP_DEVERR_CAPACITY);
+                }
             }
             bulk_commit();
-            bulk_wait_read<0>();  // the buffer is refilled after the barrier below
+            if (t + (int)gridDim.x < T) bulk_wait_read<0>();  // the buffer is refilled for the next token
         }
         if (M::kScales && !bulk_scl) {
             // MN-major scales, or scale rows that are not a multiple of 16 bytes: plain stores.
@@ -388,9 +676,23 @@ __global__ void __launch_bounds__(32 * kRowWarps) dispatch_row_kernel(DispatchAr
         __syncthreads();
     }
 
-    const int n_pad = ld_cg(a.num_pad_rows);
+    if (!laid_out) row_layout_count(la, L, ev, w0);  // a CTA with no token (padding rows only)
+
+    // Padding rows, one thread per row, slice by slice from the zero buffer.
+    const int n_pad = kLayout ? L.padoff[la.h.num_experts] : ld_cg(a.num_pad_rows);
     for (int p = blockIdx.x * blockDim.x + tid; p < n_pad; p += gridDim.x * blockDim.x) {
-        const int row = ld_cg(a.pad_rows + p);
+        int row;
+        if (kLayout) {
+            row = row_pad_row(L, la.h.num_experts, p);
+            la.h.pad_rows[p] = row;
+            if (row < a.max_rows) {
+                la.h.recv_src[row] = -1;
+                if (la.recv_topk_idx) la.recv_topk_idx[row] = -1;
+                if (la.recv_topk_weights) la.recv_topk_weights[row] = 0.0f;
+            }
+        } else {
+            row = ld_cg(a.pad_rows + p);
+        }
         if (row < 0 || row >= a.max_rows) {
             if (row >= a.max_rows) atomicOr(a.error_word, EP_DEVERR_CAPACITY);
             continue;
@@ -411,31 +713,33 @@ __global__ void __launch_bounds__(32 * kRowWarps) dispatch_row_kernel(DispatchAr
                     store_scale<kMode>(a, row, b, nullptr, 0, keep);
         }
     }
+    if (kLayout) row_totals(la, L);
     pdl_launch_dependents();
     bulk_wait_all();
 }
 
-template <int kMode>
-cudaError_t launch_row_t(const DispatchArgs& a, cudaStream_t stream) {
+template <int kMode, bool kLayout, typename IdxT>
+cudaError_t launch_row_t(const DispatchArgs& a, const LayoutArgs& la, cudaStream_t stream) {
     const SliceGeo g = slice_geo(kMode, a.H);
-    const size_t smem = row_smem_bytes(g);
-    auto kernel = dispatch_row_kernel<kMode>;
+    const size_t smem =
+        row_smem_bytes(g) + (kLayout ? row_layout_bytes(a.T * a.k, la.h.num_experts) : 0);
+    auto kernel = dispatch_row_kernel<kMode, kLayout, IdxT>;
     cudaError_t err;
     if (smem > 48 * 1024) {
         err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (err != cudaSuccess) return err;
     }
     int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 32 * kRowWarps, smem);
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kRowThreads, smem);
     if (err != cudaSuccess) return err;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int64_t cap = (int64_t)device_sm_count() * per_sm;
     int64_t want = a.T;
-    const int64_t pad_ctas = ((int64_t)a.max_pad_rows + 32 * kRowWarps - 1) / (32 * kRowWarps);
+    const int64_t pad_ctas = ((int64_t)a.max_pad_rows + kRowThreads - 1) / kRowThreads;
     if (pad_ctas > want) want = pad_ctas;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(want < 1 ? 1 : (want < cap ? want : cap)));
-    cfg.blockDim = dim3(32 * kRowWarps);
+    cfg.blockDim = dim3(kRowThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -443,8 +747,15 @@ cudaError_t launch_row_t(const DispatchArgs& a, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    debug_launch("dispatch_row_kernel", kMode, cfg);
-    return cudaLaunchKernelEx(&cfg, kernel, a);
+    debug_launch(kLayout ? "dispatch_row_kernel(layout)" : "dispatch_row_kernel", kMode, cfg);
+    return cudaLaunchKernelEx(&cfg, kernel, a, la);
+}
+
+// Whether a dispatch of this shape takes the row path: at most one layout
+// chunk of slots, no SM budget, and a row buffer that fits.
+bool row_path(const DispatchArgs& a, int mode) {
+    return (int64_t)a.T * a.k <= kLayoutChunkSlots && sm_budget() == 0 &&
+           row_smem_bytes(slice_geo(mode, a.H)) <= kRowSmemMax;
 }
 
 template <int kMode, int kW>
@@ -487,14 +798,34 @@ template <int kMode>
 cudaError_t launch_t(const DispatchArgs& a, cudaStream_t stream) {
     const int budget = sm_budget();
     if (budget > 0) return launch_w<kMode, kBudgetWarps>(a, budget, stream);
-    if ((int64_t)a.T * a.k <= kLayoutChunkSlots && row_smem_bytes(slice_geo(kMode, a.H)) <= kRowSmemMax)
-        return launch_row_t<kMode>(a, stream);
+    if (row_path(a, kMode)) return launch_row_t<kMode, false, int>(a, LayoutArgs{}, stream);
     return launch_w<kMode, kWarps>(a, 0, stream);
+}
+
+template <int kMode>
+cudaError_t launch_fused_m(const LayoutArgs& la, const DispatchArgs& a, bool idx_is_int64, cudaStream_t stream) {
+    return idx_is_int64 ? launch_row_t<kMode, true, long long>(a, la, stream)
+                        : launch_row_t<kMode, true, int>(a, la, stream);
 }
 
 }  // namespace
 
 size_t dispatch_smem_bytes(ep_x_mode mode, int H) { return smem_bytes(slice_geo(mode, H), kBudgetWarps); }
+
+cudaError_t launch_layout_dispatch_fused(const LayoutArgs& la, const DispatchArgs& a, ep_x_mode mode,
+                                         bool idx_is_int64, cudaStream_t stream) {
+    if (la.num_chunks != 1 || !row_path(a, mode) ||
+        row_smem_bytes(slice_geo(mode, a.H)) + row_layout_bytes(a.T * a.k, la.h.num_experts) >
+            kRowSmemMax)
+        return cudaErrorNotSupported;
+    switch (mode) {
+        case EP_X_BF16: return launch_fused_m<EP_X_BF16>(la, a, idx_is_int64, stream);
+        case EP_X_FP8: return launch_fused_m<EP_X_FP8>(la, a, idx_is_int64, stream);
+        case EP_X_BF16_TO_FP8: return launch_fused_m<EP_X_BF16_TO_FP8>(la, a, idx_is_int64, stream);
+        case EP_X_BF16_TO_NVFP4: return launch_fused_m<EP_X_BF16_TO_NVFP4>(la, a, idx_is_int64, stream);
+    }
+    return cudaErrorInvalidValue;
+}
 
 cudaError_t launch_dispatch(const DispatchArgs& a, ep_x_mode mode, cudaStream_t stream) {
     switch (mode) {

@@ -266,7 +266,7 @@ ep_status prepare_dispatch(const ep_handle* h, ep_x_mode mode, const void* x, co
     if (mode == EP_X_FP8 && h->num_tokens > 0 && (x_scales == nullptr || !aligned(x_scales, 4)))
         return invalid("x_scales must be non-NULL and 4-byte aligned for pre-quantised x");
     if (ep::dispatch_smem_bytes(mode, H) > ep::kMaxDispatchSmem)
-        return invalid("hidden %d is too large for this mode (row buffers exceed shared memory)", H);
+        return invalid("hidden %d: the dispatch stages exceed shared memory", H);
     a->x = x;
     a->x_scales = x_scales;
     a->recv_x = recv_x;
@@ -344,10 +344,15 @@ EP_API ep_status ep_layout_dispatch(ep_handle* h, const void* topk_idx, int32_t 
     if (st != EP_OK) return st;
     st = prepare_dispatch(h, mode, x, x_scales, H, recv_x, recv_scales, &da);
     if (st != EP_OK) return st;
-    // The dispatch launches while the layout runs and loads its x rows before
-    // waiting for it (x_ready); only the routing is read after the wait.
+    // One layout chunk (e.g. decode): one grid, each CTA computing the layout
+    // it needs.  Otherwise the dispatch launches while the layout runs and
+    // loads its x rows before waiting for it (x_ready); only the routing is
+    // read after the wait.
+    cudaError_t err = ep::launch_layout_dispatch_fused(la, da, mode, idx_is_int64 == 1, (cudaStream_t)stream);
+    if (err == cudaSuccess) return ok();
+    if (err != cudaErrorNotSupported) return cuda_failed("layout + dispatch launch", err);
     da.x_ready = 1;
-    cudaError_t err = ep::launch_layout(la, idx_is_int64 == 1, (cudaStream_t)stream);
+    err = ep::launch_layout(la, idx_is_int64 == 1, (cudaStream_t)stream);
     if (err != cudaSuccess) return cuda_failed("layout launch", err);
     err = ep::launch_dispatch(da, mode, (cudaStream_t)stream);
     if (err != cudaSuccess) return cuda_failed("dispatch launch", err);

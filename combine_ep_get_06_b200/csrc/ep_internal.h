@@ -61,6 +61,12 @@ constexpr size_t kMaxDispatchSmem = 200 * 1024;
 
 cudaError_t launch_dispatch(const DispatchArgs& a, ep_x_mode mode, cudaStream_t stream);
 
+// Layout and dispatch in one grid (every CTA computing the layout it needs)
+// when the slots fit one layout chunk and the row path applies;
+// cudaErrorNotSupported otherwise, with nothing launched.
+cudaError_t launch_layout_dispatch_fused(const LayoutArgs& la, const DispatchArgs& a, ep_x_mode mode,
+                                         bool idx_is_int64, cudaStream_t stream);
+
 struct CombineArgs {
     const void* y;
     const float* topk_weights;       // nullable: unweighted

@@ -85,6 +85,13 @@ EDGE = [
     (2049, 1, 3, 1, 5, 1024, "fp8_quant", 1.0),      # every slot dropped
     (131072, 8, 256, 8, 128, 128, "fp8_quant", 0.01),  # 1M slots: 1024 layout chunks
     (65536, 8, 1024, 32, 16, 64, "bf16", 0.0),        # 512 chunks x 1024 experts
+    # the dispatch's slices of 1024 elements: many slices, a short last slice,
+    # each on the warp-unit path (T*k > 1024) and on the row path (T*k <= 1024)
+    (300, 4, 32, 4, 8, 16512, "fp8_quant", 0.05),   # 17 slices, the last of 128 elements
+    (60, 4, 32, 4, 8, 16512, "fp8_quant", 0.05),    # row path: a 16.5 KB row buffer
+    (600, 3, 16, 2, 4, 9224, "bf16", 0.0),          # bf16: 10 slices, the last of 8 elements
+    (90, 3, 16, 2, 4, 9224, "bf16", 0.0),           # row path
+    (700, 2, 16, 4, 1, 24, "bf16", 0.1),            # a single slice of 24 elements (3 lanes)
 ]
 
 
