@@ -470,6 +470,7 @@ __device__ __forceinline__ void row_layout_count(const LayoutArgs& la, const Row
     if (tid < la.h.num_topk) L.w0[tid] = w0;
     __syncthreads();  // the counts are zero
     const int first = blockIdx.x * la.h.num_topk;  // the CTA's first slot
+    const bool has_token = (int)blockIdx.x < la.h.num_tokens;
     bool bad = false;
 #pragma unroll
     for (int r = 0; r < kSlotsPerThread; ++r) {
@@ -482,7 +483,7 @@ __device__ __forceinline__ void row_layout_count(const LayoutArgs& la, const Row
             L.eidx[i] = e;
             if (e >= 0) {
                 atomicAdd(&L.cnt[e], 1);
-                if (i < first) atomicAdd(&L.pre[e], 1);
+                if (has_token && i < first) atomicAdd(&L.pre[e], 1);
             }
         }
     }
@@ -538,14 +539,18 @@ __device__ __forceinline__ void row_slots(const LayoutArgs& la, const RowLayout&
     }
 }
 
-// Every CTA's share of the handle totals: the per-expert arrays of experts
-// [E*b/G, E*(b+1)/G), and the token counts of segments g = b, b+G, ... (a
-// token counts once in each segment one of its valid slots reaches; block
-// sum of the threads' counts).  CTA 0 also writes offsets[E] and the
-// padding count.
+// The handle totals, in shares.  When the grid has CTAs without a token row
+// (blockIdx.x >= T), those alone take the shares, so that the token CTAs
+// end with their row copies; otherwise every CTA takes one.  Share b of G:
+// the per-expert arrays of experts [E*b/G, E*(b+1)/G), and the token
+// counts of segments g = b, b+G, ... (a token counts once in each segment
+// one of its valid slots reaches; block sum of the threads' counts).
+// Share 0 also writes offsets[E] and the padding count.
 __device__ __forceinline__ void row_totals(const LayoutArgs& la, const RowLayout& L) {
     const int E = la.h.num_experts, S = la.h.num_segments, k = la.h.num_topk, T = la.h.num_tokens;
-    const int b = blockIdx.x, G = gridDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tb = (int)gridDim.x > T ? T : 0;  // the first CTA with a share
+    if ((int)blockIdx.x < tb) return;          // CTA-uniform
+    const int b = blockIdx.x - tb, G = gridDim.x - tb, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int e0 = (int)((int64_t)E * b / G), e1 = (int)((int64_t)E * (b + 1) / G);
     for (int e = e0 + tid; e < e1; e += kRowThreads) {
         la.h.counts[e] = L.cnt[e];
@@ -718,6 +723,8 @@ __global__ void __launch_bounds__(kRowThreads, 2) dispatch_row_kernel(DispatchAr
     bulk_wait_all();
 }
 
+constexpr int kTotalsCtas = 8;
+
 template <int kMode, bool kLayout, typename IdxT>
 cudaError_t launch_row_t(const DispatchArgs& a, const LayoutArgs& la, cudaStream_t stream) {
     const SliceGeo g = slice_geo(kMode, a.H);
@@ -734,7 +741,9 @@ cudaError_t launch_row_t(const DispatchArgs& a, const LayoutArgs& la, cudaStream
     if (err != cudaSuccess) return err;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int64_t cap = (int64_t)device_sm_count() * per_sm;
-    int64_t want = a.T;
+    // With the layout: up to kTotalsCtas more CTAs than tokens take the
+    // handle totals (row_totals), on SMs the token CTAs leave free.
+    int64_t want = a.T + (kLayout ? std::min(la.h.num_segments, kTotalsCtas) : 0);
     const int64_t pad_ctas = ((int64_t)a.max_pad_rows + kRowThreads - 1) / kRowThreads;
     if (pad_ctas > want) want = pad_ctas;
     cudaLaunchConfig_t cfg = {};
