@@ -436,6 +436,23 @@ __device__ __forceinline__ long long ld_idx(const IdxT* p) {
         return v;
     }
 }
+// The four consecutive indices of a thread in 16-byte loads (p 16-byte
+// aligned): fewer load instructions and L2 requests for the same bytes,
+// which every CTA of the grid reads.
+template <typename IdxT>
+__device__ __forceinline__ void ld_idx4(const IdxT* p, long long (&v)[4]) {
+    if constexpr (sizeof(IdxT) == 8) {
+        asm volatile("ld.global.nc.v2.s64 {%0, %1}, [%2];" : "=l"(v[0]), "=l"(v[1]) : "l"(p));
+        asm volatile("ld.global.nc.v2.s64 {%0, %1}, [%2];" : "=l"(v[2]), "=l"(v[3]) : "l"(p + 2));
+    } else {
+        int a, b, c, d;
+        asm volatile("ld.global.nc.v4.s32 {%0, %1, %2, %3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "l"(p));
+        v[0] = a;
+        v[1] = b;
+        v[2] = c;
+        v[3] = d;
+    }
+}
 __device__ __forceinline__ float ld_weight(const float* p) {
     float v;
     asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
@@ -449,10 +466,16 @@ __device__ __forceinline__ void row_layout_load(const LayoutArgs& la, const RowL
                                                 long long (&ev)[kSlotsPerThread], float& w0) {
     const int E = la.h.num_experts, n = la.h.num_tokens * la.h.num_topk;
     const int tid = threadIdx.x;
+    static_assert(kSlotsPerThread == 4, "ld_idx4 loads four slots");
+    const int i0 = tid * kSlotsPerThread;
+    if (i0 + kSlotsPerThread <= n && (reinterpret_cast<uintptr_t>(la.topk_idx) & 15) == 0) {
+        ld_idx4((const IdxT*)la.topk_idx + i0, ev);
+    } else {
 #pragma unroll
-    for (int r = 0; r < kSlotsPerThread; ++r) {
-        const int i = tid * kSlotsPerThread + r;
-        ev[r] = i < n ? ld_idx((const IdxT*)la.topk_idx + i) : -1;
+        for (int r = 0; r < kSlotsPerThread; ++r) {
+            const int i = i0 + r;
+            ev[r] = i < n ? ld_idx((const IdxT*)la.topk_idx + i) : -1;
+        }
     }
     w0 = 0.0f;
     if (tid < la.h.num_topk && la.topk_weights && (int)blockIdx.x < la.h.num_tokens)

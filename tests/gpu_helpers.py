@@ -155,11 +155,18 @@ def max_bf16_ulp_diff(a_bits: np.ndarray, b_bits: np.ndarray) -> int:
     return int(np.abs(ordered(a_bits) - ordered(b_bits)).max(initial=0))
 
 
-def run_cuda_one_call(inp: dict, w: W.Workload, mode: int, *, prequant=None):
+def run_cuda_one_call(inp: dict, w: W.Workload, mode: int, *, prequant=None, idx_dtype=torch.int64,
+                      idx_shift=0):
     """layout + dispatch through one ep.dispatch(x, topk_idx, ...) call;
-    returns host arrays like run_cuda (no combine)."""
+    returns host arrays like run_cuda (no combine).  idx_dtype: int64 or
+    int32 indices; idx_shift: elements by which topk_idx starts past a
+    256-byte aligned allocation (1 gives a pointer that is not 16-byte
+    aligned)."""
     T = inp["x"].shape[0]
-    idx = torch.from_numpy(inp["topk_idx"]).cuda()
+    src = torch.from_numpy(inp["topk_idx"]).to(idx_dtype)
+    base = torch.empty(src.numel() + idx_shift, dtype=idx_dtype, device="cuda")
+    idx = base[idx_shift:].view(src.shape)
+    idx.copy_(src.cuda())
     wts = torch.from_numpy(inp["topk_weights"]).cuda()
     handle = ep.EPHandle(T, w.k, w.E, w.S, w.align, device="cuda")
     rows = handle.max_recv_rows
