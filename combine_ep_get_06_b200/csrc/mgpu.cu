@@ -13,12 +13,15 @@
 // ascending slots), goes to row first_e + slot_map[s] - offsets[e] of rank
 // e/(E/W).  Warp units, as in the one-GPU dispatch: a unit is 1024
 // elements of one token row (or one of this rank's padding rows).  The warp
-// loads and converts the slice into its shared-memory stage, then copies it
-// with 16-byte stores to the slice's k destinations: peers' blocks through
-// the peer table, as plain stores over NVLink.  The warp that takes a
-// token's first slice also writes the token's slot metadata.  Padding rows
-// are zeroed in this rank's own block, and CTA 0 writes its receive totals.
-// No barrier after the tables: warps never wait on one another.
+// keeps its next unit's x loads and routing loads in flight, converts the
+// slice into one of its kStages shared-memory stages, and lanes j < k copy
+// the stage to the slice's k destinations in peers' blocks (through the
+// peer table) with TMA bulk copies, shared -> global, never multicast.
+// Where a destination is not 16-byte aligned the warp stores it with plain
+// stores instead.  The warp that takes a token's first slice also writes
+// the token's slot metadata.  Padding rows are zeroed in this rank's own
+// block from a zero buffer, and CTA 0 writes its receive totals.  No
+// barrier after the tables: warps never wait on one another.
 
 // Combine.  The one-GPU combine with rows (rank, row) from dest: y is
 // loaded from the owners' blocks.  The arithmetic is the same: fp32 FMA
@@ -37,6 +40,7 @@ constexpr int kThreads = 256;
 
 constexpr int kWarps = kThreads / 32;
 constexpr int kMinUnitsPerWarp = 8;
+constexpr int kStages = 4;  // shared-memory stages per warp
 
 struct MgpuSmem {
     int* first;      // [E]
@@ -46,7 +50,8 @@ struct MgpuSmem {
     int* own_off;    // [epr]
     int* padoff;     // [epr + 1]
     char** peer;     // [W]
-    unsigned char* stages;  // [kWarps][stage_bytes]
+    unsigned char* zeros;   // [stage_bytes] of zeros
+    unsigned char* stages;  // [kWarps][kStages][stage_bytes]
 };
 
 __host__ __device__ inline size_t align16(size_t n) { return (n + 15) & ~(size_t)15; }
@@ -66,7 +71,8 @@ __host__ __device__ inline size_t mgpu_smem(int E, int epr, int W, int stage_byt
     unsigned char* own_off = take((size_t)epr * 4);
     unsigned char* padoff = take((size_t)(epr + 1) * 4);
     unsigned char* peer = take((size_t)W * sizeof(char*));
-    unsigned char* stages = take((size_t)kWarps * stage_bytes);
+    unsigned char* zeros = take((size_t)stage_bytes);
+    unsigned char* stages = take((size_t)kWarps * kStages * stage_bytes);
     if (m != nullptr) {
         m->first = (int*)first;
         m->lofs = (int*)lofs;
@@ -75,6 +81,7 @@ __host__ __device__ inline size_t mgpu_smem(int E, int epr, int W, int stage_byt
         m->own_off = (int*)own_off;
         m->padoff = (int*)padoff;
         m->peer = (char**)peer;
+        m->zeros = zeros;
         m->stages = stages;
     }
     return at;
@@ -177,8 +184,46 @@ __device__ __forceinline__ void warp_zero_out(char* dst, int n, int lane) {
     }
 }
 
+// The raw routing loads of unit u, issued a unit ahead: per lane j < k the
+// slot's local row and expert (and on a token's first slice its weight);
+// for pre-quantised FP8 the slice's block scales.
+struct Route {
+    int lr;
+    long long e;
+    float w;
+    float xs;
+};
+
 template <int kMode>
-__global__ void __launch_bounds__(kThreads, 3) mgpu_dispatch_kernel(MgpuArgs a) {
+__device__ __forceinline__ Route load_route(const MgpuArgs& a, const SliceGeo& sg, int64_t u, int64_t n_tok_units,
+                                            int lane) {
+    Route r;
+    r.lr = -1;
+    r.e = -1;
+    r.w = 0.0f;
+    r.xs = 0.0f;
+    if (u >= n_tok_units) return r;
+    const int k = a.g.num_topk;
+    const int t = (int)(u / sg.ns), s = (int)(u - (int64_t)t * sg.ns);
+    if (lane < k) {
+        const size_t sl = (size_t)t * k + lane;
+        r.lr = a.slot_map[sl];
+        r.e = a.idx_is_int64 ? ((const int64_t*)a.topk_idx)[sl] : ((const int32_t*)a.topk_idx)[sl];
+        if (s == 0 && a.topk_weights) r.w = a.topk_weights[sl];
+    }
+    if (kMode == EP_X_FP8) {
+        const int ne = min(kSliceElems, a.g.hidden - s * kSliceElems);
+        if (lane < ne / 128) r.xs = a.src.x_scales[(size_t)t * (a.g.hidden / 128) + s * (kSliceElems / 128) + lane];
+    }
+    return r;
+}
+
+__device__ __forceinline__ bool bulk_ok(const void* dst, int n) {
+    return ((reinterpret_cast<uintptr_t>(dst) | (uintptr_t)n) & 15) == 0;
+}
+
+template <int kMode>
+__global__ void __launch_bounds__(kThreads, 2) mgpu_dispatch_kernel(MgpuArgs a) {
     using M = Mode<kMode>;
     extern __shared__ __align__(128) unsigned char smem[];
     const ep_mgpu_geometry& g = a.g;
@@ -190,10 +235,19 @@ __global__ void __launch_bounds__(kThreads, 3) mgpu_dispatch_kernel(MgpuArgs a) 
     const int rb_bytes = g.row_bytes, sc_bytes = g.scale_bytes;
     uint32_t* const err = (uint32_t*)(a.local_block + g.off_error_word);
     int2* const dest = (int2*)(a.local_block + g.off_dest);
-    unsigned char* const st = m.stages + (size_t)warp * sg.stage_bytes;
-    unsigned char* const sst = st + sg.out_bytes;
+    unsigned char* const stages = m.stages + (size_t)warp * kStages * sg.stage_bytes;
 
-    build_tables(a, m);
+    // The first unit's loads fly while the tables are built (the grid
+    // starts after the layout and the counts exchange have completed).
+    const int64_t n_tok_units = (int64_t)T * sg.ns;
+    const int64_t stride = (int64_t)gridDim.x * kWarps;
+    int64_t u = (int64_t)blockIdx.x * kWarps + warp;
+    Loads<kMode> nxt = load_x<kMode>(a.src, sg, u, n_tok_units, lane);
+    Route nrt = load_route<kMode>(a, sg, u, n_tok_units, lane);
+
+    for (int i = tid; i < sg.stage_bytes / 16; i += kThreads) reinterpret_cast<uint4*>(m.zeros)[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+    build_tables(a, m);  // ends with a barrier
     const int n_pad = m.padoff[epr];
 
     if (blockIdx.x == 0) {
@@ -211,9 +265,16 @@ __global__ void __launch_bounds__(kThreads, 3) mgpu_dispatch_kernel(MgpuArgs a) 
         }
     }
 
-    const int64_t n_tok_units = (int64_t)T * sg.ns;
     const int64_t n_units = n_tok_units + n_pad;
-    for (int64_t u = (int64_t)blockIdx.x * kWarps + warp; u < n_units; u += (int64_t)gridDim.x * kWarps) {
+    int it = 0;  // token units of this warp (selects the stage)
+    for (; u < n_units; u += stride) {
+        const Loads<kMode> cur = nxt;
+        const Route rt = nrt;
+        {
+            const int64_t un = u + stride;
+            nxt = load_x<kMode>(a.src, sg, un, n_tok_units, lane);
+            nrt = load_route<kMode>(a, sg, un, n_tok_units, lane);
+        }
         if (u >= n_tok_units) {
             // one of this rank's padding rows, in its own block
             const int p = (int)(u - n_tok_units);
@@ -223,8 +284,25 @@ __global__ void __launch_bounds__(kThreads, 3) mgpu_dispatch_kernel(MgpuArgs a) 
                 if (lane == 0) atomicOr(err, EP_DEVERR_CAPACITY);
                 continue;
             }
-            warp_zero_out(a.local_block + g.off_recv_x + (size_t)row * rb_bytes, rb_bytes, lane);
-            if (sc_bytes > 0) warp_zero_out(a.local_block + g.off_recv_scales + (size_t)row * sc_bytes, sc_bytes, lane);
+            char* const dx = a.local_block + g.off_recv_x + (size_t)row * rb_bytes;
+            char* const ds = a.local_block + g.off_recv_scales + (size_t)row * sc_bytes;
+            bool plain_x = false, plain_s = false;
+            for (int s = lane; s < sg.ns; s += 32) {
+                const int ne = min(kSliceElems, g.hidden - s * kSliceElems);
+                const int db = ne * sg.out_bytes / kSliceElems;
+                char* const px = dx + (size_t)s * sg.out_bytes;
+                if (bulk_ok(px, db)) bulk_s2g(px, m.zeros, db);
+                else plain_x = true;
+                if (sc_bytes > 0) {
+                    const int sb = ne / M::kScaleBlock * M::kScaleBytes;
+                    char* const ps = ds + (size_t)s * sg.sout_bytes;
+                    if (bulk_ok(ps, sb)) bulk_s2g(ps, m.zeros, sb);
+                    else plain_s = true;
+                }
+            }
+            bulk_commit();
+            if (__any_sync(0xffffffffu, plain_x)) warp_zero_out(dx, rb_bytes, lane);
+            if (__any_sync(0xffffffffu, plain_s)) warp_zero_out(ds, sc_bytes, lane);
             if (lane == 0) {
                 ((int32_t*)(a.local_block + g.off_recv_src))[row] = -1;
                 ((int32_t*)(a.local_block + g.off_recv_topk_idx))[row] = -1;
@@ -233,29 +311,20 @@ __global__ void __launch_bounds__(kThreads, 3) mgpu_dispatch_kernel(MgpuArgs a) 
             continue;
         }
 
-        // A token slice: its loads first, so they fly while the routing resolves.
+        // A token slice: resolve its routing (loaded a unit ago).
         const int t = (int)(u / sg.ns), s = (int)(u - (int64_t)t * sg.ns);
         const int ne = min(kSliceElems, g.hidden - s * kSliceElems);
-        const Loads<kMode> l = load_x<kMode>(a.src, sg, u, n_tok_units, lane);
-        Meta mt;
-        mt.row = -1;
-        mt.xs = 0.0f;
-        if (kMode == EP_X_FP8 && lane < ne / 128)
-            mt.xs = a.src.x_scales[(size_t)t * (g.hidden / 128) + s * (kSliceElems / 128) + lane];
         int d = -1, row = -1;
         if (lane < k) {
             const size_t sl = (size_t)t * k + lane;
-            const int lr = a.slot_map[sl];
-            if (lr >= 0) {
-                const int64_t e64 =
-                    a.idx_is_int64 ? ((const int64_t*)a.topk_idx)[sl] : ((const int32_t*)a.topk_idx)[sl];
-                const int e = (int)e64;
-                if (e64 < 0 || e64 >= g.num_experts) {
+            if (rt.lr >= 0) {
+                if (rt.e < 0 || rt.e >= g.num_experts) {
                     // not the topk_idx the layout saw: drop the slot
                     if (s == 0) atomicOr(err, EP_DEVERR_BAD_TOPK_IDX);
                 } else {
+                    const int e = (int)rt.e;
                     d = e / epr;
-                    row = m.first[e] + (lr - m.lofs[e]);
+                    row = m.first[e] + (rt.lr - m.lofs[e]);
                 }
                 if (d < 0) {
                     row = -1;
@@ -265,30 +334,62 @@ __global__ void __launch_bounds__(kThreads, 3) mgpu_dispatch_kernel(MgpuArgs a) 
                 } else if (s == 0) {
                     char* pb = m.peer[d];
                     ((int32_t*)(pb + g.off_recv_src))[row] = (int32_t)((int64_t)g.rank * g.max_tokens * k + sl);
-                    ((int32_t*)(pb + g.off_recv_topk_idx))[row] = e;
-                    ((float*)(pb + g.off_recv_topk_weights))[row] = a.topk_weights ? a.topk_weights[sl] : 0.0f;
+                    ((int32_t*)(pb + g.off_recv_topk_idx))[row] = (int)rt.e;
+                    ((float*)(pb + g.off_recv_topk_weights))[row] = rt.w;
                 }
             }
             if (s == 0) dest[sl] = make_int2(d, row);
         }
-        __syncwarp();  // the previous unit's copies have read the stage
-        fill_stage<kMode>(l, mt, ne, lane, st, sst);
+
+        unsigned char* const st = stages + (size_t)(it % kStages) * sg.stage_bytes;
+        unsigned char* const sst = st + sg.out_bytes;
+        ++it;
+        // The copies issued from this stage kStages units ago must have read it.
+        if (lane < k) bulk_wait_read<kStages - 1>();
+        __syncwarp();
+        Meta mt;
+        mt.row = -1;
+        mt.xs = rt.xs;
+        fill_stage<kMode>(cur, mt, ne, lane, st, sst);
+        fence_proxy_async_smem();
         __syncwarp();
         const int db = ne * sg.out_bytes / kSliceElems;
         const int sb = M::kScales ? ne / M::kScaleBlock * M::kScaleBytes : 0;
-        for (int j = 0; j < k; ++j) {
+        bool plain_x = false, plain_s = false;
+        if (lane < k) {
+            if (d >= 0) {
+                char* const pb = m.peer[d];
+                char* const px = pb + g.off_recv_x + (size_t)row * rb_bytes + (size_t)s * sg.out_bytes;
+                if (bulk_ok(px, db)) bulk_s2g(px, st, db);
+                else plain_x = true;
+                if (sb > 0) {
+                    char* const ps = pb + g.off_recv_scales + (size_t)row * sc_bytes + (size_t)s * sg.sout_bytes;
+                    if (bulk_ok(ps, sb)) bulk_s2g(ps, sst, sb);
+                    else plain_s = true;
+                }
+            }
+            bulk_commit();
+        }
+        // Destinations a bulk copy cannot take: the whole warp stores them.
+        unsigned px_mask = __ballot_sync(0xffffffffu, plain_x), ps_mask = __ballot_sync(0xffffffffu, plain_s);
+        while (px_mask | ps_mask) {
+            const int j = __ffs(px_mask | ps_mask) - 1;
             const int dj = __shfl_sync(0xffffffffu, d, j), rj = __shfl_sync(0xffffffffu, row, j);
-            if (dj < 0) continue;
-            char* pb = m.peer[dj];
-            warp_copy_out(pb + g.off_recv_x + (size_t)rj * rb_bytes + (size_t)s * sg.out_bytes, st, db, lane);
-            if (sb > 0)
+            char* const pb = m.peer[dj];
+            if (px_mask >> j & 1)
+                warp_copy_out(pb + g.off_recv_x + (size_t)rj * rb_bytes + (size_t)s * sg.out_bytes, st, db, lane);
+            if (ps_mask >> j & 1)
                 warp_copy_out(pb + g.off_recv_scales + (size_t)rj * sc_bytes + (size_t)s * sg.sout_bytes, sst, sb,
                               lane);
+            px_mask &= ~(1u << j);
+            ps_mask &= ~(1u << j);
         }
     }
-    // The CTA's stores to peers' memory are ordered before the grid's end:
-    // the barrier makes them precede thread 0's system-scope fence, which is
+    // The CTA's writes to peers' memory are ordered before the grid's end:
+    // each thread waits for its bulk copies to complete, the barrier makes
+    // all of them precede thread 0's system-scope fence, which is
     // cumulative.  (A fence in every thread measured as the top stall.)
+    bulk_wait_all();
     __syncthreads();
     if (tid == 0) __threadfence_system();
 }

@@ -252,10 +252,16 @@ class LocalRanks:
         return out
 
     def exchange_counts(self, handles: Sequence[EPHandle]):
-        """The all-gather of step 2, as device copies."""
+        """The all-gather of step 2, as device copies: one stack, then one
+        multi-tensor copy into every block (a launch each instead of one per
+        block)."""
         stacked = torch.stack([h.counts for h in handles])
-        for b in self.blocks:
-            b.all_counts.copy_(stacked)
+        dsts = [b.all_counts for b in self.blocks]
+        if hasattr(torch, "_foreach_copy_"):
+            torch._foreach_copy_(dsts, [stacked] * len(dsts))
+        else:
+            for d in dsts:
+                d.copy_(stacked)
 
     def dispatch(self, xs, topk_idxs, topk_weights=None, *, use_fp8=False, use_nvfp4=False) -> List[EPHandle]:
         handles = self._per_rank(lambda r: self.ranks[r].layout(topk_idxs[r]))
