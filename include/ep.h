@@ -226,9 +226,15 @@ EP_API ep_status ep_dispatch(const ep_handle* handle, ep_x_mode mode, const void
  * num_experts, expert_alignment) call of the DeepEP V2 README ("Interfaces
  * and examples"), which routes and sends in one step.  Arguments, results
  * and errors are those of ep_get_layout followed by ep_dispatch with the
- * same handle.  It launches the same kernels, but because it knows that the
- * dispatch directly follows the layout, the dispatch reads its x rows while
- * the layout still runs (the two calls cannot assume that). */
+ * same handle.  With more than one layout chunk of slots (T*k > 1024) it
+ * launches the same kernels, but because it knows that the dispatch
+ * directly follows the layout, the dispatch reads its x rows while the
+ * layout still runs (the two calls cannot assume that).  With at most one
+ * chunk (e.g. decode, T*k <= 1024) and no SM budget, one kernel does both:
+ * every token CTA computes in shared memory the part of the layout its row
+ * needs, and a few CTAs without a token write the handle's totals.  The
+ * workspace is then checked but not written.  The outputs are the same
+ * either way. */
 EP_API ep_status ep_layout_dispatch(ep_handle* handle, const void* topk_idx, int32_t idx_is_int64,
                                     const float* topk_weights, int32_t* recv_topk_idx,
                                     float* recv_topk_weights, void* workspace,
