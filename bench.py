@@ -558,7 +558,9 @@ def run_workload_lines(args, dev, name: str, peak: float) -> dict:
         gbs = b / (ms * 1e-3) / 1e9
         return {"us": round(ms * 1e3, 2), "bytes": b, "gbs": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4)}
 
+    in_mb = (x.numel() * x.element_size() + y.numel() * y.element_size()) / 1e6
     return {"config": step_config(w, T, 1)["workload"], "valid_rows": V, "padding_rows": P,
+            "l2": f"no flush: the step's inputs (x and y, {in_mb:.0f} MB) exceed the 126 MB L2",
             "step": line(sum(nb.values()), step_ms), "dispatch": line(nb["dispatch"], dis_ms),
             "combine": line(nb["combine"], com_ms)}
 
