@@ -386,10 +386,13 @@ __global__ void __launch_bounds__(kThreads, 2) mgpu_dispatch_kernel(MgpuArgs a) 
         }
     }
     // The CTA's writes to peers' memory are ordered before the grid's end:
-    // each thread waits for its bulk copies to complete, the barrier makes
-    // all of them precede thread 0's system-scope fence, which is
-    // cumulative.  (A fence in every thread measured as the top stall.)
+    // each thread waits for its bulk copies to complete and orders them
+    // (async proxy) before its own later accesses (proxy fence); the
+    // barrier makes all of them precede thread 0's system-scope fence,
+    // which is cumulative.  (A system fence in every thread measured as the
+    // top stall.)
     bulk_wait_all();
+    fence_proxy_async_global();
     __syncthreads();
     if (tid == 0) __threadfence_system();
 }
