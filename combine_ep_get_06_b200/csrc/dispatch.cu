@@ -244,12 +244,12 @@ __global__ void __launch_bounds__(32 * kW, kW == kWarps ? 2 : 1) dispatch_kernel
 // takes whole token rows.  Each lane converts items of 16 consecutive
 // elements (8 in bf16) into one shared row buffer -- a 1x128 block is 8
 // lanes (3 shuffles), an NVFP4 block one lane -- so a row of hidden 7168
-// takes two rounds of the CTA's threads.  After a barrier lanes j < k of
-// warp 0 copy the whole row, and its scale row, to the k receive rows with
-// one bulk copy each.  A decode launch (T=128, hidden 7168, FP8) took
-// 4.19 us in warp units, whose copies are seven times as many and a seventh
-// of the size.  Padding rows go one thread per row, slice by slice from a
-// zeroed buffer.
+// takes two rounds of the CTA's threads.  After a barrier lane 0 of warp j
+// copies the whole row, and its scale row, to the receive row of slot j
+// (j, j + 8, ...) with one bulk copy each.  A decode launch (T=128, hidden
+// 7168, FP8) took 4.19 us in warp units, whose copies are seven times as
+// many and a seventh of the size.  Padding rows go one thread per row,
+// slice by slice from a zeroed buffer.
 constexpr int kRowWarps = 8;
 constexpr int kRowThreads = 32 * kRowWarps;
 static_assert(kLayoutChunkSlots % kRowThreads == 0, "a one-chunk layout spreads evenly over a row CTA");
@@ -325,12 +325,15 @@ __host__ __device__ inline size_t row_smem_bytes(const SliceGeo& g) {
 //
 // With at most kLayoutChunkSlots slots there is no layout grid.  Every CTA
 // reads all T*k expert indices into shared memory and computes what it
-// needs: the per-expert counts (shared atomics), the aligned expert offsets
-// (a scan over the experts), and, for each slot of its own tokens, the
-// number of earlier slots with the same expert (ballot counts over the
-// index array), which gives the slot's row.  It writes the handle entries
-// of its own slots and of the padding rows it zeroes; CTA 0 also writes the
-// totals and the tokens per segment.  No CTA waits for another.
+// needs: the per-expert counts and the counts before its first token
+// (shared atomics), the aligned expert offsets (a scan over the experts),
+// and, for each slot of its tokens, the number of earlier slots with the
+// same expert (for its first token the prefix counts plus the token's own
+// earlier slots; for later ones ballot counts over the index array), which
+// gives the slot's row.  It writes the handle entries of its own slots and
+// of the padding rows it zeroes.  The handle totals (per-expert arrays,
+// tokens per segment) are written in slices by the CTAs without a token
+// row, or by all CTAs when every CTA has one.  No CTA waits for another.
 
 // Shared memory of the in-CTA layout, after the row buffers.
 struct RowLayout {
