@@ -60,6 +60,9 @@ def test_checked_build_matches_oracle_and_no_check_fires():
 def test_debug_prints_each_launch():
     r = _child({"EP_DEBUG": "1"})
     assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-3000:]
+    # mid: the layout grids and the warp-unit dispatch; decode one-call: the
+    # one-kernel layout + dispatch; tiny two-call: the one-CTA layout and
+    # the row-path dispatch
     for kernel in ("layout_count_kernel", "layout_assign_kernel", "layout_single_kernel", "dispatch_kernel",
-                   "combine_kernel"):
+                   "dispatch_row_kernel(layout)", "dispatch_row_kernel", "combine_kernel"):
         assert f"[ep] {kernel}<" in r.stderr, kernel
