@@ -220,7 +220,19 @@ __global__ void __launch_bounds__(32 * kW, kW == kWarps ? 2 : 1) dispatch_kernel
     const int64_t u = (int64_t)blockIdx.x * kW + warp;
 
     Loads<kMode> nxt;
-    if (a.x_ready) {
+    if (!a.x_ready) {
+        // x may still be written by the previous grid: only ask L2 for the
+        // first units (a prefetch returns no value, and L2 is where every
+        // write lands), and load them after the wait.
+        const int64_t up = u + (int64_t)lane * stride;
+        if (lane <= kPrefetchUnits && up < n_tok_units) {
+            const int t = (int)(up / g.ns), s = (int)(up - (int64_t)t * g.ns);
+            const int ne = min(kSliceElems, a.H - s * kSliceElems);
+            const size_t eb = kMode == EP_X_FP8 ? 1 : 2;  // input bytes per element
+            bulk_prefetch_l2((const char*)a.x + ((size_t)t * a.H + (size_t)s * kSliceElems) * eb,
+                             (uint32_t)(ne * eb));
+        }
+    } else {
         // x is complete: load the first unit and ask L2 for the next few
         // while the layout finishes.
         nxt = load_x<kMode>(a, g, u, n_tok_units, lane);

@@ -61,9 +61,18 @@ __global__ void __launch_bounds__(kThreads) layout_count_kernel(LayoutArgs a) {
     const int64_t s = (int64_t)t0 * k + tid;
     const IdxT* idx = (const IdxT*)a.topk_idx;
 
+    // The chunk's indices are asked into L2 while the previous grid still
+    // runs: a prefetch returns no value and L2 is where every write lands,
+    // so it cannot observe a stale index (the loads come after the wait).
+    // Only the 16-byte aligned interior of the chunk, never past its ends.
+    if (tid == 0) {
+        const uintptr_t lo = ((uintptr_t)(idx + (int64_t)t0 * k) + 15) & ~(uintptr_t)15;
+        const uintptr_t hi = (uintptr_t)(idx + (int64_t)t1 * k) & ~(uintptr_t)15;
+        if (hi > lo) bulk_prefetch_l2((const void*)lo, (uint32_t)(hi - lo));
+    }
     // Programmatic dependent launch: wait for the previous grid before any
-    // global access; only then let the assign pass start (it reads topk_idx
-    // before waiting on this grid).
+    // global load or store; only then let the assign pass start (it reads
+    // topk_idx before waiting on this grid).
     pdl_wait();
     pdl_launch_dependents();
     bool bad = false;
