@@ -33,6 +33,21 @@ __global__ void __launch_bounds__(kMaxT) combine_kernel(CombineArgs a, int ipr, 
     const int T = a.T, k = a.k, H = a.H;
     const char* const y = (const char*)a.y;
     const size_t row_bytes = (size_t)H * 2;
+    const int64_t n_units = (int64_t)T * upr;
+    // With more units than the grid holds at once (a persistent grid), the
+    // slot map and weights of the CTA's first units are asked into L2 while
+    // the previous grid drains: a prefetch returns no value and every write
+    // lands in L2, so nothing stale is observed (the loads come after the
+    // wait).  Only the 16-byte aligned interior of each range.  (A one-wave
+    // batch, as at decode, measured slower with it.)
+    if (tid == 0 && n_units > (int64_t)gridDim.x * nsub) {
+        const int64_t u_lo = (int64_t)blockIdx.x * nsub, u_hi = min(n_units, u_lo + nsub);
+        if (u_hi > u_lo) {
+            const int64_t s_lo = u_lo / upr * k, s_hi = ((u_hi - 1) / upr + 1) * k;
+            prefetch_interior_l2(a.slot_map + s_lo, a.slot_map + s_hi);
+            if (a.topk_weights != nullptr) prefetch_interior_l2(a.topk_weights + s_lo, a.topk_weights + s_hi);
+        }
+    }
     pdl_wait();
 
     // dispatch_backward's weight gradient: gather each slot's row value.
@@ -44,7 +59,6 @@ __global__ void __launch_bounds__(kMaxT) combine_kernel(CombineArgs a, int ipr, 
         }
     }
 
-    const int64_t n_units = (int64_t)T * upr;
     const int64_t u0 = sub < nsub ? (int64_t)blockIdx.x * nsub + sub : n_units;
     for (int64_t u = u0; u < n_units; u += (int64_t)gridDim.x * nsub) {
         const int t = (int)(u / upr);

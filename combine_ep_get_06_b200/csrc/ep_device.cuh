@@ -106,6 +106,12 @@ __device__ __forceinline__ void bulk_s2g(void* gdst, const void* ssrc, uint32_t 
 __device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
+// An L2 prefetch of the 16-byte aligned part of [lo, hi): it never reaches
+// past either end of the range.
+__device__ __forceinline__ void prefetch_interior_l2(const void* lo, const void* hi) {
+    const uintptr_t a = ((uintptr_t)lo + 15) & ~(uintptr_t)15, b = (uintptr_t)hi & ~(uintptr_t)15;
+    if (b > a) bulk_prefetch_l2((const void*)a, (uint32_t)(b - a));
+}
 
 // An L2 evict-last policy (createpolicy) and a store that takes one.
 __device__ __forceinline__ uint64_t l2_evict_last_policy() {

@@ -65,11 +65,7 @@ __global__ void __launch_bounds__(kThreads) layout_count_kernel(LayoutArgs a) {
     // runs: a prefetch returns no value and L2 is where every write lands,
     // so it cannot observe a stale index (the loads come after the wait).
     // Only the 16-byte aligned interior of the chunk, never past its ends.
-    if (tid == 0) {
-        const uintptr_t lo = ((uintptr_t)(idx + (int64_t)t0 * k) + 15) & ~(uintptr_t)15;
-        const uintptr_t hi = (uintptr_t)(idx + (int64_t)t1 * k) & ~(uintptr_t)15;
-        if (hi > lo) bulk_prefetch_l2((const void*)lo, (uint32_t)(hi - lo));
-    }
+    if (tid == 0) prefetch_interior_l2(idx + (int64_t)t0 * k, idx + (int64_t)t1 * k);
     // Programmatic dependent launch: wait for the previous grid before any
     // global load or store; only then let the assign pass start (it reads
     // topk_idx before waiting on this grid).
