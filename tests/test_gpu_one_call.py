@@ -64,10 +64,12 @@ def test_one_call_dispatch_edge_shapes(T, k, E, S, align, H, xm, drop, dup):
 
 
 @pytest.mark.parametrize("dtype,shift", [(torch.int32, 0), (torch.int32, 1), (torch.int64, 1)])
-@pytest.mark.parametrize("T", [128, 127])
+@pytest.mark.parametrize("T", [128, 127, 300])
 def test_one_call_index_types_and_alignment(T, dtype, shift):
     # the one-chunk path loads four indices a thread with 16-byte loads when
-    # the pointer allows it, else one by one; T = 127 leaves a partial group
+    # the pointer allows it, else one by one; T = 127 leaves a partial group.
+    # T = 300 (2400 slots, three chunks) takes the layout grids, whose count
+    # kernel prefetches only the 16-byte aligned interior of its chunk
     w = W.Workload("idx", T=T, H=1024, E=64, S=4, k=8, align=4, x_mode="fp8_quant")
     inp = _random_case(T, 8, 64, 4, 4, 1024, 0.1, seed=T + shift)
     g = run_cuda_one_call(inp, w, ep.EP_X_BF16_TO_FP8, idx_dtype=dtype, idx_shift=shift)
