@@ -9,7 +9,7 @@
 //     lanes, by xor shuffles; scale and inverse by IEEE division; e4m3
 //     conversion) into a per-warp shared-memory stage, and lanes j < k
 //     copy the stage to the slice of receive row slot_map[t*k+j] with TMA
-//     bulk copies (cp.async.bulk shared->global, never multicast); or
+//     bulk copies (cp.async.bulk shared->global, one destination each); or
 //   - a padding row: lanes copy a zeroed buffer over the row's slices.
 // Units are numbered token-major (t, slice), then padding rows, and dealt
 // to the warps grid-stride, so every warp gets the same mix of small units

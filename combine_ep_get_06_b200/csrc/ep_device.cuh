@@ -77,7 +77,7 @@ __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// ---- TMA bulk copies shared -> global (never multicast)
+// ---- TMA bulk copies shared -> global (one destination each)
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

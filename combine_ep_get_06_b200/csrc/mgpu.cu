@@ -16,7 +16,7 @@
 // keeps its next unit's x loads and routing loads in flight, converts the
 // slice into one of its kStages shared-memory stages, and lanes j < k copy
 // the stage to the slice's k destinations in peers' blocks (through the
-// peer table) with TMA bulk copies, shared -> global, never multicast.
+// peer table) with TMA bulk copies, shared -> global, one destination each.
 // Where a destination is not 16-byte aligned the warp stores it with plain
 // stores instead.  The warp that takes a token's first slice also writes
 // the token's slot metadata.  Padding rows are zeroed in this rank's own

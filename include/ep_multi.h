@@ -7,10 +7,11 @@
  * Here the segments of ep.h become ranks: rank d of W owns experts
  * [d*E/W, (d+1)*E/W).  Each rank holds one device "rank block" whose
  * sections have the same offsets on every rank (ep_mgpu_geometry).  Every
- * rank maps every other rank's block (CUDA IPC over NVLink / NVSwitch, no
- * multicast), and the kernels store received rows straight into the
- * owner's block and load expert outputs straight from it, with plain
- * 16-byte loads and stores.
+ * rank maps every other rank's block (CUDA IPC over NVLink / NVSwitch), and
+ * the kernels store received rows straight into the owner's block (TMA bulk
+ * copies from shared memory, one destination each; plain 16-byte stores
+ * where a destination is not 16-byte aligned) and load expert outputs
+ * straight from it with plain 16-byte loads.
  *
  * One step on rank r, with T_r <= max_tokens tokens:
  *   1. ep_get_layout on a local handle (num_segments = W, alignment 1):
@@ -98,7 +99,7 @@ EP_API ep_status ep_mgpu_geometry_init(ep_mgpu_geometry* g, int32_t rank, int32_
 EP_API ep_status ep_mgpu_block_alloc(size_t bytes, void** block);
 EP_API ep_status ep_mgpu_block_free(void* block);
 
-/* CUDA IPC of a rank block (not multicast): ep_ipc_export writes
+/* CUDA IPC of a rank block: ep_ipc_export writes
  * EP_IPC_HANDLE_BYTES bytes that another process, on this GPU or another
  * one of the node, passes to ep_ipc_import, which maps the block into that
  * process (peer access enabled lazily) and returns its address there.
