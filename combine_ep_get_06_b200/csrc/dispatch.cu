@@ -562,6 +562,8 @@ __device__ __forceinline__ void row_slots(const LayoutArgs& la, const RowLayout&
             if (row >= la.h.max_recv_rows) {
                 if (lane == 0) atomicOr(la.h.error_word, EP_DEVERR_CAPACITY);
                 row = -1;
+            } else if (!EP_CHECK(before < L.cnt[e], la.h.error_word)) {
+                row = -1;  // the rank must fall inside the expert's slots (checked builds only)
             } else if (lane == 0) {
                 la.h.recv_src[row] = s;
                 if (la.recv_topk_idx) la.recv_topk_idx[row] = e;
