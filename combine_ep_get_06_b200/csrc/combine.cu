@@ -17,7 +17,11 @@
 namespace ep {
 namespace {
 
-constexpr int kMaxThreads = 256;  // threads of a unit at most
+constexpr int kMaxThreads = 448;   // threads of a unit at most (V3: two units of 448 per token row)
+constexpr int kSmallThreads = 256; // launch bound of the kernel for units of at most this many threads
+
+// Threads of a unit under an SM budget at most (a CTA holds several).
+constexpr int kBudgetUnitThreads = 256;
 
 // Threads of a CTA under an SM budget, for k <= 8*G: as many as fit an SM
 // without spilling the k row values a thread holds.
@@ -163,14 +167,20 @@ cudaError_t launch_bd(const CombineArgs& a, int ipr, int ut, int bd, int max_cta
 template <int G>
 cudaError_t launch_t(const CombineArgs& a, cudaStream_t stream) {
     const int ipr = a.H / 8;
-    int ut = unit_threads(ipr, kMaxThreads);
     const int budget = sm_budget();
-    if (budget == 0 && (int64_t)a.T * ((ipr + ut - 1) / ut) < (int64_t)kSmallUnitsPerSm * device_sm_count())
-        ut = unit_threads(ipr, 128);
     if (budget > 0) {
+        // units of at most kBudgetUnitThreads, several to a CTA of kT threads
         constexpr int kT = budget_threads<G>();
+        const int ut = unit_threads(ipr, kBudgetUnitThreads);
         return launch_bd<G, kT>(a, ipr, ut, (kT / ut) * ut, budget, stream);
     }
+    int ut = unit_threads(ipr, kMaxThreads);
+    if ((int64_t)a.T * ((ipr + ut - 1) / ut) < (int64_t)kSmallUnitsPerSm * device_sm_count())
+        ut = unit_threads(ipr, 128);
+    // Units of up to 256 threads keep the kernel built for 256-thread
+    // blocks: the looser bound of the 448-thread build lets the compiler
+    // take registers that cost those launches an SM's worth of occupancy.
+    if (ut <= kSmallThreads) return launch_bd<G, kSmallThreads>(a, ipr, ut, ut, 0, stream);
     return launch_bd<G, kMaxThreads>(a, ipr, ut, ut, 0, stream);
 }
 

@@ -92,6 +92,10 @@ EDGE = [
     (600, 3, 16, 2, 4, 9224, "bf16", 0.0),          # bf16: 10 slices, the last of 8 elements
     (90, 3, 16, 2, 4, 9224, "bf16", 0.0),           # row path
     (700, 2, 16, 4, 1, 24, "bf16", 0.1),            # a single slice of 24 elements (3 lanes)
+    # the combine's unit sizes: two 448-thread units a row with k > 8 (two slot
+    # groups), and 128-thread units for a one-wave batch
+    (200, 12, 64, 4, 8, 7168, "bf16", 0.1),
+    (24, 12, 64, 4, 8, 7168, "fp8_quant", 0.1),
 ]
 
 
