@@ -256,15 +256,27 @@ __global__ void __launch_bounds__(32 * kW, kW == kWarps ? 2 : 1) dispatch_kernel
 // takes whole token rows.  Each lane converts items of 16 consecutive
 // elements (8 in bf16) into one shared row buffer -- a 1x128 block is 8
 // lanes (3 shuffles), an NVFP4 block one lane -- so a row of hidden 7168
-// takes two rounds of the CTA's threads.  After a barrier lane 0 of warp j
-// copies the whole row, and its scale row, to the receive row of slot j
-// (j, j + 8, ...) with one bulk copy each.  A decode launch (T=128, hidden
+// takes two rounds of the CTA's threads (one in the 16-warp CTAs of the
+// one-kernel layout path).  After a barrier lane 0 of warp j copies the
+// whole row, and its scale row, to the receive row of slot j (j, j + the
+// CTA's warps, ...) with one bulk copy each.  A decode launch (T=128, hidden
 // 7168, FP8) took 4.19 us in warp units, whose copies are seven times as
 // many and a seventh of the size.  Padding rows go one thread per row,
 // slice by slice from a zeroed buffer.
 constexpr int kRowWarps = 8;
-constexpr int kRowThreads = 32 * kRowWarps;
-static_assert(kLayoutChunkSlots % kRowThreads == 0, "a one-chunk layout spreads evenly over a row CTA");
+// The one-kernel layout + dispatch takes 16-warp CTAs (one to an SM): a
+// decode row converts in one round and the layout steps spread over twice
+// the threads (the cached-handle launch measured faster with 8 warps).
+constexpr int kLayoutWarps = 16;
+constexpr int kLayoutThreads = 32 * kLayoutWarps;
+static_assert(kLayoutChunkSlots % kLayoutThreads == 0, "a one-chunk layout spreads evenly over a CTA");
+
+template <bool kLayout>
+struct RowShape {
+    static constexpr int kWarps = kLayout ? kLayoutWarps : kRowWarps;
+    static constexpr int kThreads = 32 * kWarps;
+    static constexpr int kMinBlocks = kLayout ? 1 : 2;  // CTAs per SM the registers allow for
+};
 constexpr size_t kRowSmemMax = 96 * 1024;
 
 template <int kMode>
@@ -354,7 +366,7 @@ struct RowLayout {
     int* pre;     // [E]   slots of each expert before the CTA's first token
     int* off;     // [E+1] first row of each expert
     int* padoff;  // [E+1] first padding index of each expert
-    int* wsum;    // [2*kRowWarps] scan of the warps' sums
+    int* wsum;    // [2*kLayoutWarps] scan of the warps' sums
     float* w0;    // [kMaxTopk] weights of the CTA's first token's slots
     __device__ RowLayout(int* p, int n, int E) {
         eidx = p;
@@ -363,20 +375,20 @@ struct RowLayout {
         off = pre + E;
         padoff = off + E + 1;
         wsum = padoff + E + 1;
-        w0 = reinterpret_cast<float*>(wsum + 2 * kRowWarps);
+        w0 = reinterpret_cast<float*>(wsum + 2 * kLayoutWarps);
     }
 };
 
 __host__ __device__ inline size_t row_layout_bytes(int n, int E) {
-    return sizeof(int) * ((size_t)n + 2 * (size_t)E + 2 * ((size_t)E + 1) + 2 * kRowWarps + kMaxTopk);
+    return sizeof(int) * ((size_t)n + 2 * (size_t)E + 2 * ((size_t)E + 1) + 2 * kLayoutWarps + kMaxTopk);
 }
 
 // off / padoff from cnt: aligned rows A(c) = ceil(c/a)*a and padding rows
-// A(c) - c, scanned over the experts by kRowThreads threads, each taking a
+// A(c) - c, scanned over the experts by kLayoutThreads threads, each taking a
 // run of consecutive experts.  Barriers inside; ends with one.
 __device__ __forceinline__ void row_expert_offsets(const RowLayout& L, int E, int align) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int per = (E + kRowThreads - 1) / kRowThreads;
+    const int per = (E + kLayoutThreads - 1) / kLayoutThreads;
     const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
     int r = 0, p = 0;
     for (int e = e0; e < e1; ++e) {
@@ -395,13 +407,13 @@ __device__ __forceinline__ void row_expert_offsets(const RowLayout& L, int E, in
     }
     if (lane == 31) {
         L.wsum[warp] = ri;
-        L.wsum[kRowWarps + warp] = pi;
+        L.wsum[kLayoutWarps + warp] = pi;
     }
     __syncthreads();
     int rb = ri - r, pb = pi - p;
     for (int w = 0; w < warp; ++w) {
         rb += L.wsum[w];
-        pb += L.wsum[kRowWarps + w];
+        pb += L.wsum[kLayoutWarps + w];
     }
     for (int e = e0; e < e1; ++e) {
         const int c = L.cnt[e], re = align == 1 ? c : (c + align - 1) / align * align;
@@ -410,7 +422,7 @@ __device__ __forceinline__ void row_expert_offsets(const RowLayout& L, int E, in
         rb += re;
         pb += re - c;
     }
-    if (tid == kRowThreads - 1) {
+    if (tid == kLayoutThreads - 1) {
         L.off[E] = rb;
         L.padoff[E] = pb;
     }
@@ -434,7 +446,7 @@ __device__ __forceinline__ int row_pad_row(const RowLayout& L, int E, int p) {
 // and of the weights of the CTA's first token, and zeroes the counts;
 // row_layout_count then (after a barrier) stores the indices, counts them
 // per expert (and before the CTA's first token), and scans the offsets.
-constexpr int kSlotsPerThread = kLayoutChunkSlots / kRowThreads;
+constexpr int kSlotsPerThread = kLayoutChunkSlots / kLayoutThreads;
 
 // An index load issued where it stands (a volatile asm is not moved past
 // the other volatile loads), so that it is in flight during the conversion.
@@ -451,21 +463,18 @@ __device__ __forceinline__ long long ld_idx(const IdxT* p) {
         return v;
     }
 }
-// The four consecutive indices of a thread in 16-byte loads (p 16-byte
-// aligned): fewer load instructions and L2 requests for the same bytes,
-// which every CTA of the grid reads.
+// The two consecutive indices of a thread in one vector load (p aligned to
+// the pair: 16 bytes for int64, 8 for int32): fewer load instructions and
+// L2 requests for the same bytes, which every CTA of the grid reads.
 template <typename IdxT>
-__device__ __forceinline__ void ld_idx4(const IdxT* p, long long (&v)[4]) {
+__device__ __forceinline__ void ld_idx2(const IdxT* p, long long (&v)[2]) {
     if constexpr (sizeof(IdxT) == 8) {
         asm volatile("ld.global.nc.v2.s64 {%0, %1}, [%2];" : "=l"(v[0]), "=l"(v[1]) : "l"(p));
-        asm volatile("ld.global.nc.v2.s64 {%0, %1}, [%2];" : "=l"(v[2]), "=l"(v[3]) : "l"(p + 2));
     } else {
-        int a, b, c, d;
-        asm volatile("ld.global.nc.v4.s32 {%0, %1, %2, %3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "l"(p));
+        int a, b;
+        asm volatile("ld.global.nc.v2.s32 {%0, %1}, [%2];" : "=r"(a), "=r"(b) : "l"(p));
         v[0] = a;
         v[1] = b;
-        v[2] = c;
-        v[3] = d;
     }
 }
 __device__ __forceinline__ float ld_weight(const float* p) {
@@ -481,10 +490,10 @@ __device__ __forceinline__ void row_layout_load(const LayoutArgs& la, const RowL
                                                 long long (&ev)[kSlotsPerThread], float& w0) {
     const int E = la.h.num_experts, n = la.h.num_tokens * la.h.num_topk;
     const int tid = threadIdx.x;
-    static_assert(kSlotsPerThread == 4, "ld_idx4 loads four slots");
+    static_assert(kSlotsPerThread == 2, "ld_idx2 loads two slots");
     const int i0 = tid * kSlotsPerThread;
-    if (i0 + kSlotsPerThread <= n && (reinterpret_cast<uintptr_t>(la.topk_idx) & 15) == 0) {
-        ld_idx4((const IdxT*)la.topk_idx + i0, ev);
+    if (i0 + kSlotsPerThread <= n && (reinterpret_cast<uintptr_t>(la.topk_idx) % (2 * sizeof(IdxT))) == 0) {
+        ld_idx2((const IdxT*)la.topk_idx + i0, ev);
     } else {
 #pragma unroll
         for (int r = 0; r < kSlotsPerThread; ++r) {
@@ -495,7 +504,7 @@ __device__ __forceinline__ void row_layout_load(const LayoutArgs& la, const RowL
     w0 = 0.0f;
     if (tid < la.h.num_topk && la.topk_weights && (int)blockIdx.x < la.h.num_tokens)
         w0 = ld_weight(la.topk_weights + (size_t)blockIdx.x * la.h.num_topk + tid);
-    for (int e = tid; e < E; e += kRowThreads) {
+    for (int e = tid; e < E; e += kLayoutThreads) {
         L.cnt[e] = 0;
         L.pre[e] = 0;
     }
@@ -531,13 +540,13 @@ __device__ __forceinline__ void row_layout_count(const LayoutArgs& la, const Row
 }
 
 // The rows of token t's slots into rows_s, and their handle entries.  Slot
-// j is warp j % kRowWarps's: its row is off[e] plus the number of earlier
+// j is warp j % kLayoutWarps's: its row is off[e] plus the number of earlier
 // slots (flat order) with expert e.  For the CTA's first token that is
 // pre[e] plus the token's own earlier slots; for later ones (several tokens
 // to a CTA) the slots are counted 128 at a time by ballots.
 __device__ __forceinline__ void row_slots(const LayoutArgs& la, const RowLayout& L, int t, int* rows_s) {
     const int k = la.h.num_topk, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int j = warp; j < k; j += kRowWarps) {
+    for (int j = warp; j < k; j += kLayoutWarps) {
         const int s = t * k + j;
         const int e = L.eidx[s];
         int row = -1;
@@ -592,7 +601,7 @@ __device__ __forceinline__ void row_totals(const LayoutArgs& la, const RowLayout
     if ((int)blockIdx.x < tb) return;          // CTA-uniform
     const int b = blockIdx.x - tb, G = gridDim.x - tb, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int e0 = (int)((int64_t)E * b / G), e1 = (int)((int64_t)E * (b + 1) / G);
-    for (int e = e0 + tid; e < e1; e += kRowThreads) {
+    for (int e = e0 + tid; e < e1; e += kLayoutThreads) {
         la.h.counts[e] = L.cnt[e];
         la.h.recv_counts[e] = L.off[e + 1] - L.off[e];
         la.h.offsets[e] = L.off[e];
@@ -605,7 +614,7 @@ __device__ __forceinline__ void row_totals(const LayoutArgs& la, const RowLayout
     for (int gs = b; gs < S; gs += G) {
         const int lo = gs * per_seg, hi = lo + per_seg;  // the segment's experts
         int c = 0;
-        for (int t = tid; t < T; t += kRowThreads) {
+        for (int t = tid; t < T; t += kLayoutThreads) {
             bool has = false;
             for (int j = 0; j < k; ++j) {
                 const int e = L.eidx[t * k + j];
@@ -620,7 +629,7 @@ __device__ __forceinline__ void row_totals(const LayoutArgs& la, const RowLayout
         __syncthreads();
         if (tid == 0) {
             int sum = 0;
-            for (int w = 0; w < kRowWarps; ++w) sum += L.wsum[w];
+            for (int w = 0; w < kLayoutWarps; ++w) sum += L.wsum[w];
             la.h.seg_tokens[gs] = sum;
         }
     }
@@ -630,7 +639,9 @@ __device__ __forceinline__ void row_totals(const LayoutArgs& la, const RowLayout
 // grid of ep_layout_dispatch, so x too is read only after the wait);
 // otherwise the routing comes from the handle the layout grid wrote.
 template <int kMode, bool kLayout, typename IdxT>
-__global__ void __launch_bounds__(kRowThreads, 2) dispatch_row_kernel(DispatchArgs a, LayoutArgs la) {
+__global__ void __launch_bounds__(RowShape<kLayout>::kThreads, RowShape<kLayout>::kMinBlocks)
+    dispatch_row_kernel(DispatchArgs a, LayoutArgs la) {
+    constexpr int kW = RowShape<kLayout>::kWarps, kT = RowShape<kLayout>::kThreads;
     using M = Mode<kMode>;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ int rows_s[kMaxTopk];
@@ -645,10 +656,10 @@ __global__ void __launch_bounds__(kRowThreads, 2) dispatch_row_kernel(DispatchAr
     char* const rscl = (char*)a.recv_scales;
     const int k = a.k, T = a.T;
     const uint64_t keep = a.scales_ld > 0 ? l2_evict_last_policy() : 0;
-    zero_buffer<kRowWarps>(zeros, g.stage_bytes);
+    zero_buffer<kW>(zeros, g.stage_bytes);
     __syncthreads();
 
-    // The thread's items of a row are c = warp*32 + lane + j*kRowThreads,
+    // The thread's items of a row are c = warp*32 + lane + j*kT,
     // taken two at a time with both loads issued first.  The first pair of
     // the CTA's first row is loaded before the wait when x is already
     // complete (directly after the layout grid).
@@ -658,12 +669,12 @@ __global__ void __launch_bounds__(kRowThreads, 2) dispatch_row_kernel(DispatchAr
     const bool first_ok = blockIdx.x < (unsigned)T;
     if (a.x_ready && first_ok) {
         fa = row_load<kMode>(a, blockIdx.x, c0 + lane, c0 + lane < ipr);
-        fb = row_load<kMode>(a, blockIdx.x, c0 + kRowThreads + lane, c0 + kRowThreads + lane < ipr);
+        fb = row_load<kMode>(a, blockIdx.x, c0 + kT + lane, c0 + kT + lane < ipr);
     }
     pdl_wait();
     if (!a.x_ready && first_ok) {
         fa = row_load<kMode>(a, blockIdx.x, c0 + lane, c0 + lane < ipr);
-        fb = row_load<kMode>(a, blockIdx.x, c0 + kRowThreads + lane, c0 + kRowThreads + lane < ipr);
+        fb = row_load<kMode>(a, blockIdx.x, c0 + kT + lane, c0 + kT + lane < ipr);
     }
     bool have_first = first_ok && c0 < ipr;  // used by the first pass of the loop below
     long long ev[kSlotsPerThread];
@@ -674,8 +685,8 @@ __global__ void __launch_bounds__(kRowThreads, 2) dispatch_row_kernel(DispatchAr
     const bool bulk_scl = M::kScales && a.bulk_scales;
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
         if (!kLayout && tid < k) rows_s[tid] = ld_cg(a.slot_map + (size_t)t * k + tid);
-        for (int c = c0; c < ipr; c += 2 * kRowThreads) {
-            const int ca = c + lane, cb = c + kRowThreads + lane;
+        for (int c = c0; c < ipr; c += 2 * kT) {
+            const int ca = c + lane, cb = c + kT + lane;
             Item2 ia, ib;
             if (have_first) {
                 ia = fa;
@@ -686,7 +697,7 @@ __global__ void __launch_bounds__(kRowThreads, 2) dispatch_row_kernel(DispatchAr
                 ib = row_load<kMode>(a, t, cb, cb < ipr);
             }
             row_fill<kMode>(a, t, ca, ca < ipr, ia, rowbuf, sclbuf);
-            if (c + kRowThreads < ipr) row_fill<kMode>(a, t, cb, cb < ipr, ib, rowbuf, sclbuf);
+            if (c + kT < ipr) row_fill<kMode>(a, t, cb, cb < ipr, ib, rowbuf, sclbuf);
         }
         if (kLayout) {
             if (!laid_out) {
@@ -697,8 +708,8 @@ __global__ void __launch_bounds__(kRowThreads, 2) dispatch_row_kernel(DispatchAr
         }
         fence_proxy_async_smem();
         __syncthreads();
-        if (lane == 0) {  // warp j issues the copies of slots j, j + kRowWarps, ...
-            for (int j = warp; j < k; j += kRowWarps) {
+        if (lane == 0) {  // warp j issues the copies of slots j, j + kW, ...
+            for (int j = warp; j < k; j += kW) {
                 const int row = rows_s[j];
                 if (row >= 0 && row < a.max_rows) {
                     bulk_s2g(recv + (size_t)row * g.row_bytes, rowbuf, g.row_bytes);
@@ -777,18 +788,18 @@ cudaError_t launch_row_t(const DispatchArgs& a, const LayoutArgs& la, cudaStream
         if (err != cudaSuccess) return err;
     }
     int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kRowThreads, smem);
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, RowShape<kLayout>::kThreads, smem);
     if (err != cudaSuccess) return err;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int64_t cap = (int64_t)device_sm_count() * per_sm;
     // With the layout: up to kTotalsCtas more CTAs than tokens take the
     // handle totals (row_totals), on SMs the token CTAs leave free.
     int64_t want = a.T + (kLayout ? std::min(la.h.num_segments, kTotalsCtas) : 0);
-    const int64_t pad_ctas = ((int64_t)a.max_pad_rows + kRowThreads - 1) / kRowThreads;
+    const int64_t pad_ctas = ((int64_t)a.max_pad_rows + RowShape<kLayout>::kThreads - 1) / RowShape<kLayout>::kThreads;
     if (pad_ctas > want) want = pad_ctas;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(want < 1 ? 1 : (want < cap ? want : cap)));
-    cfg.blockDim = dim3(kRowThreads);
+    cfg.blockDim = dim3(RowShape<kLayout>::kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
